@@ -1,0 +1,347 @@
+"""Paged-attention decode benchmark: GB/s (and % of HBM peak) and decode tokens/s per step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload b256] [--impl ours|reference]
+
+A step is one pass of the hot path over one batch: reshape_and_cache of the
+step's new K/V rows, then paged decode attention over every sequence (and,
+for the mixed workload, the chunked-prefill kernel).  ``value`` is the
+algorithmic bytes of the step (K/V read by decode, q/out, block tables, the
+rows written by reshape_and_cache) over the device time of the step, summed
+over ranks.  With N > 1 (torchrun) every rank runs its own replica of the
+workload on its own GPU (weak scaling, no collective on the data path); the
+time is the max over ranks.
+
+``--impl reference`` times the float64 CPU oracle on the host cores instead
+(a bounded sample of the same workload per step); under torchrun only rank 0
+runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth_inputs as si  # noqa: E402
+
+METRIC = "paged-attn decode GB/s (% of B200 HBM peak) and decode tokens/s at 1 GPU"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def step_bytes(w, seq_lens, tables_cols, n_step_rows):
+    """Algorithmic bytes of one step (see the module docstring)."""
+    H, D, bs = w.num_heads, w.head_dim, w.block_size
+    lens = np.asarray(seq_lens, dtype=np.int64)
+    kv = int(lens.sum()) * H * D * 2 * 2
+    qo = 2 * len(lens) * H * D * 2
+    meta = int(((lens + bs - 1) // bs).sum()) * 4 + len(lens) * 4
+    reshape = n_step_rows * H * D * 2 * 2 * 2 + n_step_rows * 8
+    decode = kv + qo + meta
+    prefill = 0
+    if w.prefill is not None:
+        L, c = w.prefill.chunk, w.prefill.ctx_before
+        prefill = (c + L) * H * D * 2 * 2 + 2 * L * H * D * 2
+    return decode, reshape, prefill
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            parts = [x.strip() for x in l.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_max_sum(value_max, value_sum, device):
+    """Max of the first value and sum of the second over all ranks (identity at N = 1)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value_max, value_sum
+    t = torch.tensor([value_max], dtype=torch.float64, device=device)
+    u = torch.tensor([value_sum], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+def oracle_sample_seqs(w, budget_tokens):
+    """A seeded sample of decode sequences whose context totals about budget_tokens."""
+    rng = np.random.default_rng(1234)
+    order = rng.permutation(w.num_seqs)
+    pick, tot = [], 0
+    for s in order:
+        if pick and tot + w.decode_lens[s] > budget_tokens:
+            continue
+        pick.append(int(s))
+        tot += w.decode_lens[s]
+        if tot >= budget_tokens:
+            break
+    return sorted(pick)
+
+
+def time_oracle(w, steps, warmup, budget_tokens):
+    """Times the CPU oracle's decode on a bounded sample; returns (GB/s, s/step, sample desc, threads)."""
+    from oracle import attention as oatt
+    from oracle import workloads as owl
+    sample = oracle_sample_seqs(w, budget_tokens)
+    o = owl.build(w, seqs=sample)
+    kc, vc = o.k_cache, o.v_cache
+    oatt.reshape_and_cache(kc, vc, o.k_step, o.v_step, o.slot_mapping, w.block_size)
+    idx = np.asarray(sample)
+    args = (o.q[idx], kc, vc, o.block_tables[idx], o.seq_lens[idx], w.block_size, w.scale)
+    for _ in range(warmup):
+        oatt.paged_attention_decode(*args)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oatt.paged_attention_decode(*args)
+    dt = (time.perf_counter() - t0) / steps
+    nbytes = int(o.seq_lens[idx].astype(np.int64).sum()) * w.num_heads * w.head_dim * 4
+    threads = _blas_threads()
+    desc = (f"oracle float64 decode of {len(sample)} of {w.num_seqs} sequences "
+            f"({int(o.seq_lens[idx].sum())} cached tokens), GB/s scaled by their K/V bytes")
+    return nbytes / dt / 1e9, dt, desc, threads
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    w = si.get(args.workload)
+    gbs, dt, desc, threads = time_oracle(w, args.steps, args.warmup, args.oracle_tokens)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": 0,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "num_seqs": w.num_seqs, "num_heads": w.num_heads, "head_dim": w.head_dim,
+                   "block_size": w.block_size, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_cache_411_b200 as pk
+    from paged_kv_cache_411_b200 import workload as pwl
+
+    world, rank, local = dist_setup()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    w = si.get(args.workload)
+    ds = pwl.build(w, device=device)
+    S, H, D = ds.q.shape
+    T = ds.k_step.shape[0]
+    ws = torch.empty(pk.decode_workspace_bytes(S, H, D, ds.max_blocks, w.block_size), dtype=torch.uint8,
+                     device=device)
+    out = torch.empty_like(ds.q)
+    pout = torch.empty_like(ds.prefill_q) if ds.prefill_q is not None else None
+    stream = torch.cuda.current_stream(device)
+    dec_b, rs_b, pre_b = step_bytes(w, ds.seq_lens_host, ds.max_blocks, T)
+    step_b = dec_b + rs_b + pre_b
+
+    def step(ev=None):
+        pk.reshape_and_cache(ds.k_step, ds.v_step, ds.k_cache, ds.v_cache, ds.slot_mapping, stream=stream)
+        if pout is not None:
+            pk.paged_attention_prefill_chunk(pout, ds.prefill_q, ds.k_cache, ds.v_cache, ds.prefill_table,
+                                             ds.prefill_q_start, ds.prefill_ctx_before, w.scale, stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        pk.paged_attention_decode(out, ds.q, ds.k_cache, ds.v_cache, ds.block_tables, ds.seq_lens, w.scale, ws,
+                                  stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+
+    dec_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        time.sleep(0.25)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(device)
+        t0.record(stream)
+        for i in range(args.steps):
+            step(dec_events[i])
+        t1.record(stream)
+        torch.cuda.synchronize(device)
+        if world > 1:
+            dist.barrier()
+    local_ms = t0.elapsed_time(t1)
+    dec_ms = [a.elapsed_time(b) for a, b in dec_events]
+    total_ms, total_bytes = reduce_max_sum(local_ms, step_b * args.steps, device)
+    ms_per_step = total_ms / args.steps
+    value = total_bytes / (total_ms / 1e3) / 1e9
+    peak, peak_kind = measured_peaks()
+
+    # end to end: pinned host inputs -> device, the step, the output back to the host, every step
+    host = {k: getattr(ds, k).cpu().pin_memory() for k in ("q", "k_step", "v_step", "slot_mapping",
+                                                           "block_tables", "seq_lens")}
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = host_out.numel() * host_out.element_size()
+
+    def e2e_step():
+        for k, t in host.items():
+            getattr(ds, k).copy_(t, non_blocking=True)
+        step()
+        host_out.copy_(out, non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    if world > 1:
+        dist.barrier()
+    t_a = time.perf_counter()
+    for _ in range(args.steps):
+        e2e_step()
+    e2e_s = time.perf_counter() - t_a
+    e2e_max, e2e_bytes = reduce_max_sum(e2e_s, step_b * args.steps, device)
+    e2e_value = e2e_bytes / e2e_max / 1e9
+
+    if rank == 0:
+        dec_avg_ms = float(np.mean(dec_ms))
+        dec_gbs = dec_b / (dec_avg_ms / 1e3) / 1e9
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "config": {
+                "workload": w.name, "num_seqs": S, "num_heads": H, "head_dim": D, "block_size": w.block_size,
+                "context_tokens": int(ds.seq_lens_host.sum()), "step_rows_written": T,
+                "bytes_per_step": step_b, "accumulate": "f32",
+                "l2": f"inputs larger than L2 ({dec_b / 1e9:.2f} GB of K/V per step), no flush",
+                "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+            },
+            "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+            "pct_of_nominal_8tbs": round(100 * value / world / 8000.0, 2),
+            "decode_tokens_per_s": round(S * world / (ms_per_step / 1e3), 1),
+            "decode_tokens_per_s_32_layers": round(S * world / (32 * ms_per_step / 1e3), 1),
+            "roofline": {"kernel": "paged_attention_decode (plan + streaming kernel + combine)", "bound": "hbm",
+                         "achieved": round(dec_gbs, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": round(dec_gbs / peak, 4), "traffic": None,
+                         "algorithmic_bytes_per_launch": dec_b, "avg_launch_ms": round(dec_avg_ms, 5)},
+            "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": round(1e3 * e2e_max / args.steps, 4)},
+            "gpu_launches": args.steps * (4 + (1 if pout is not None else 0)),
+            "clocks": clk.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            gbs, dt, desc, threads = time_oracle(w, 1, 0, args.oracle_tokens)
+            line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                                    "sample": desc}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="b256", choices=sorted(si.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--oracle-tokens", type=int, default=12000,
+                    help="cached tokens in the oracle's bounded sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,251 @@
+/*
+ * pagedkv.h -- C ABI of libpagedkv.so: paged-KV attention for NVIDIA B200 (sm_100a).
+ *
+ * The method is PagedAttention with iteration-level (continuous) batching as
+ * described on the page "LLM 推理引擎 Continuous Batching 与 PagedAttention：
+ * 从 vLLM 原理到生产级部署实战" (cited below as [CB-PA]) and in the chapter
+ * "动态批处理算法：连续批处理、In-flight 请求管理与 PagedAttention" ([DB]).
+ * The KV cache of every request is stored in fixed-size physical blocks of
+ * `block_size` tokens taken from one shared pool; a per-request block table
+ * maps logical block i to a physical block ([CB-PA] §3.1-§3.2, [DB] §4.3).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every function returns a pa_status; nothing is thrown across the ABI.
+ *   On an error the message of the calling thread's last error is available
+ *   from pa_last_error().
+ * - Device entry points take DEVICE pointers that the caller allocated and
+ *   owns; the library never allocates, frees or retains device memory, and
+ *   never synchronises.  Kernels are enqueued on `stream` (a cudaStream_t
+ *   passed as void*; NULL = the legacy default stream) on the current device.
+ *   Argument errors are detected on the host before anything is enqueued.
+ * - fp16 buffers (pa_half) hold IEEE-754 binary16 values.  Arithmetic inside
+ *   the attention kernels is fp32; outputs are rounded to fp16 (nearest even).
+ * - The KV cache is two separate tensors, K and V, each laid out
+ *   [num_blocks, block_size, num_heads, head_dim] row-major (a token's heads
+ *   are contiguous inside its row, as the pointer arithmetic
+ *   "+ head_idx * head_dim" of [CB-PA] §3.3 places them).
+ * - A slot names one token row of the pool: slot = block * block_size + row.
+ * - `err_flag` (nullable, device int32): kernels check every block id, slot
+ *   and length they read from device memory; a bad one is skipped (never
+ *   dereferenced) and the matching PA_DEVCHK_* bit is OR-ed into *err_flag.
+ *   The caller reads the flag after synchronising; pa_check_device_flag()
+ *   turns a read-back value into PA_ERR_DEVICE_CHECK.
+ * - Supported kernel instances: head_dim 64 or 128; block_size 8 or a
+ *   multiple of 16; num_heads a multiple of 4 (or of 2 with head_dim 128).
+ *   Anything else returns PA_ERR_UNSUPPORTED.
+ * - The block allocator is host-only, single-threaded (one scheduler thread
+ *   owns it, as in [CB-PA] §2.2) and owned by the library from
+ *   pa_alloc_create to pa_alloc_destroy.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t pa_status;
+enum {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,   /* bad pointer, size, shape or id range            */
+    PA_ERR_OOM = 2,           /* not enough free blocks ([CB-PA] §3.2 "return False") */
+    PA_ERR_NOT_FOUND = 3,     /* unknown request id                               */
+    PA_ERR_EXISTS = 4,        /* request id already has a block table             */
+    PA_ERR_UNSUPPORTED = 5,   /* head_dim / block_size / head count not built     */
+    PA_ERR_CUDA = 6,          /* a CUDA call failed; see pa_last_error()          */
+    PA_ERR_DEVICE_CHECK = 7   /* a device-side check fired (see err_flag)         */
+};
+
+/* Bits a kernel ORs into *err_flag. */
+enum {
+    PA_DEVCHK_BLOCK_ID = 1,   /* block-table entry outside [0, num_blocks)        */
+    PA_DEVCHK_SLOT = 2,       /* slot >= num_blocks * block_size                  */
+    PA_DEVCHK_SEQ_LEN = 4,    /* seq_len < 0 or > max_blocks * block_size         */
+    PA_DEVCHK_QUERY_RANGE = 8, /* q_start not non-decreasing or past num_tokens   */
+    PA_DEVCHK_TIMEOUT = 16     /* an internal bounded wait ran out (a library bug) */
+};
+
+typedef uint16_t pa_half;
+typedef struct pa_alloc pa_alloc;
+
+typedef struct {
+    int32_t num_blocks;
+    int32_t block_size;
+    int32_t num_free;        /* blocks on the free list                             */
+    int32_t num_used;        /* blocks with refcount > 0                            */
+    int64_t total_refs;      /* sum of refcounts = sum of block-table lengths       */
+    int64_t num_requests;    /* requests with a block table                         */
+    int64_t oom_count;       /* calls that returned PA_ERR_OOM                      */
+    int64_t waste_tokens;    /* sum over requests of blocks*block_size - seq_len    */
+} pa_alloc_stats_t;
+
+/* ---- library ------------------------------------------------------------ */
+
+/* ABI version of this header (bumped on any signature change). */
+int32_t pa_abi_version(void);
+/* Message of the calling thread's last failed call ("" if none). */
+const char* pa_last_error(void);
+/* Static name of a status code. */
+const char* pa_status_string(pa_status s);
+/* PA_OK if `flag_value` (a read-back err_flag) is 0, else PA_ERR_DEVICE_CHECK. */
+pa_status pa_check_device_flag(int32_t flag_value);
+
+/* ---- host block allocator ([CB-PA] §3.2 BlockManager, §4.1 shared prefix) --
+ *
+ * Free list: starts as init_free_order (or 0..num_blocks-1 when NULL); every
+ * take pops from its END; blocks whose refcount drops to zero are pushed on
+ * the end in block-table order.  A request's block table lists its physical
+ * blocks in logical order; its seq_len counts the tokens it stores; it always
+ * holds exactly ceil(seq_len / block_size) blocks.  The allocator is not
+ * thread-safe. */
+
+/* Create a pool of `num_blocks` blocks of `block_size` tokens.
+ * init_free_order: NULL, or a permutation of 0..num_blocks-1 (host, copied).
+ * Errors: INVALID_ARG (num_blocks < 0, block_size <= 0, not a permutation, out NULL). */
+pa_status pa_alloc_create(int32_t num_blocks, int32_t block_size,
+                          const int32_t* init_free_order, pa_alloc** out);
+/* Destroy the allocator (NULL is accepted). */
+void pa_alloc_destroy(pa_alloc* a);
+
+/* [CB-PA] §3.2 allocate: give `req` a table of ceil(num_tokens / block_size)
+ * popped blocks and seq_len = num_tokens.  All-or-nothing.
+ * Errors: EXISTS (req has a table), OOM (too few free blocks; nothing changes),
+ * INVALID_ARG (num_tokens < 0). */
+pa_status pa_alloc_allocate(pa_alloc* a, int64_t req, int32_t num_tokens);
+
+/* [CB-PA] §3.2 append_token: store one more token.  With current_len the
+ * tokens stored before the call, a block is popped iff current_len %
+ * block_size == 0.  *slot_out (nullable) = slot of position current_len.
+ * Errors: NOT_FOUND, OOM (nothing changes). */
+pa_status pa_alloc_append_token(pa_alloc* a, int64_t req, int64_t* slot_out);
+
+/* n appends as one all-or-nothing step (same pops, same slots as n calls of
+ * pa_alloc_append_token).  slots_out: NULL or host int64[n].
+ * Errors: NOT_FOUND, OOM (nothing changes), INVALID_ARG (n < 0). */
+pa_status pa_alloc_append_tokens(pa_alloc* a, int64_t req, int32_t n, int64_t* slots_out);
+
+/* [CB-PA] §4.1 shared prefix: `dst` gets the first floor(prefix_tokens /
+ * block_size) blocks of `src` (whole blocks only; each refcount + 1) and
+ * seq_len = that many full blocks of tokens.  Later appends to either go to
+ * private blocks.
+ * Errors: NOT_FOUND (src), EXISTS (dst), INVALID_ARG (prefix_tokens < 0 or
+ * > seq_len(src)). */
+pa_status pa_alloc_fork(pa_alloc* a, int64_t src, int64_t dst, int32_t prefix_tokens);
+
+/* [CB-PA] §3.2 free: decrement the refcount of every block of req's table in
+ * order; push the ones reaching zero.  Freeing an unknown id is a no-op (PA_OK). */
+pa_status pa_alloc_free(pa_alloc* a, int64_t req);
+
+/* Copy req's block table into out[0..cap).  *len_out (nullable) = its length.
+ * Errors: NOT_FOUND, INVALID_ARG (cap < length; nothing copied). */
+pa_status pa_alloc_get_block_table(const pa_alloc* a, int64_t req, int32_t* out,
+                                   int32_t cap, int32_t* len_out);
+
+/* *out = seq_len(req).  Errors: NOT_FOUND, INVALID_ARG (out NULL). */
+pa_status pa_alloc_seq_len(const pa_alloc* a, int64_t req, int32_t* out);
+
+/* Slot mapping ([CB-PA] §3.3 address form): slots_out[i] = table[p / block_size]
+ * * block_size + p % block_size for p = pos_begin + i, i < n (host int64[n]).
+ * Errors: NOT_FOUND, INVALID_ARG (range outside 0..seq_len). */
+pa_status pa_alloc_slots(const pa_alloc* a, int64_t req, int32_t pos_begin, int32_t n,
+                         int64_t* slots_out);
+
+/* Pack the tables of reqs[0..n) into host int32 tables[n][max_blocks]
+ * (padding -1) and seq_lens[n], the form the kernels read.
+ * Errors: NOT_FOUND, INVALID_ARG (a table longer than max_blocks; nothing written). */
+pa_status pa_alloc_pack(const pa_alloc* a, const int64_t* reqs, int32_t n, int32_t max_blocks,
+                        int32_t* tables, int32_t* seq_lens);
+
+/* Counters (see pa_alloc_stats_t). */
+pa_status pa_alloc_stats(const pa_alloc* a, pa_alloc_stats_t* out);
+/* *out = refcount of physical block `block`.  Errors: INVALID_ARG. */
+pa_status pa_alloc_refcount(const pa_alloc* a, int32_t block, int32_t* out);
+/* Copy the free list (bottom to top; the next pop takes the last entry).
+ * Errors: INVALID_ARG (cap < length; *len_out still set). */
+pa_status pa_alloc_free_list(const pa_alloc* a, int32_t* out, int32_t cap, int32_t* len_out);
+
+/* ---- device kernels -------------------------------------------------------- */
+
+/* reshape_and_cache: write the step's new K/V rows into the pool.
+ * For t < num_tokens with s = slot_mapping[t] >= 0:
+ *   k_cache[s / block_size][s % block_size][h][d] = k_new[t][h][d]   (same for V)
+ * Tokens with a negative slot are padding and skipped.  Bit-exact copy.
+ * k_new, v_new: device fp16 [num_tokens][num_heads][head_dim].
+ * k_cache, v_cache: device fp16 [num_blocks][block_size][num_heads][head_dim].
+ * slot_mapping: device int64 [num_tokens].  Slots >= num_blocks*block_size are
+ * skipped and flagged PA_DEVCHK_SLOT.  Rows of k_new/v_new and of the cache
+ * must be 16-byte aligned (num_heads*head_dim*2 % 16 == 0).
+ * Source: the slots come from append_token ([CB-PA] §3.2) and are the
+ * addresses the attention kernel reads ([CB-PA] §3.3).
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+pa_status pa_reshape_and_cache(const pa_half* k_new, const pa_half* v_new,
+                               pa_half* k_cache, pa_half* v_cache,
+                               const int64_t* slot_mapping, int32_t num_tokens,
+                               int32_t num_heads, int32_t head_dim, int32_t block_size,
+                               int32_t num_blocks, int32_t* err_flag, void* stream);
+
+/* Bytes of device workspace pa_paged_attention_decode needs for `num_seqs`
+ * sequences whose block tables have `max_blocks` columns.  0 on bad arguments. */
+size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t head_dim,
+                                 int32_t max_blocks, int32_t block_size);
+
+/* Decode attention over the paged cache ([CB-PA] §3.3 paged_attention_kernel,
+ * completed with its omitted weighted sum of V; §1.1 decode phase).
+ * For every sequence s < num_seqs and head h:
+ *   n = seq_lens[s] (including the token decoded in this step, whose K/V must
+ *   already be in the cache); position j < n lives in physical block
+ *   block_tables[s][j / block_size] at row j % block_size;
+ *   out[s][h] = sum_j softmax_j(scale * q[s][h] . K_j[h]) V_j[h].
+ * A sequence with n == 0 gets zeros.  Table entries at or beyond
+ * ceil(n / block_size) are never read (they may hold anything).
+ * out, q: device fp16 [num_seqs][num_heads][head_dim] (16-byte aligned).
+ * k_cache, v_cache: as above (16-byte aligned base).
+ * block_tables: device int32 [num_seqs][max_blocks]; seq_lens: device int32 [num_seqs].
+ * workspace: device, >= pa_decode_workspace_bytes(num_seqs, num_heads, head_dim,
+ * max_blocks, block_size) bytes, 256-byte aligned, caller-owned scratch whose
+ * contents need no initialisation and are clobbered; two launches in flight
+ * at once must not share it.
+ * The work is split flash-decoding style into partitions of the sequence
+ * combined with the exact log-sum-exp rule, so the result does not depend on
+ * the physical placement of the blocks (bitwise) and matches a float64
+ * reference to about 1e-3.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+pa_status pa_paged_attention_decode(pa_half* out, const pa_half* q,
+                                    const pa_half* k_cache, const pa_half* v_cache,
+                                    const int32_t* block_tables, const int32_t* seq_lens,
+                                    int32_t num_seqs, int32_t num_heads, int32_t head_dim,
+                                    int32_t block_size, int32_t max_blocks, int32_t num_blocks,
+                                    float scale, void* workspace, size_t workspace_bytes,
+                                    int32_t* err_flag, void* stream);
+
+/* Chunked-prefill attention over the paged cache ([CB-PA] §4.3 Chunked
+ * Prefill; §1.1 prefill phase).  Request b < num_reqs owns query rows
+ * q_start[b] .. q_start[b+1]-1 (host-unknown, device int32 [num_reqs+1],
+ * q_start[0] = 0, non-decreasing, q_start[num_reqs] <= num_tokens); its row i
+ * sits at absolute position p = ctx_before[b] + i and attends causally to
+ * positions 0..p of its own sequence through block_tables[b]:
+ *   out[row][h] = sum_{j<=p} softmax_j(scale * q[row][h] . K_j[h]) V_j[h].
+ * The chunk's own K/V must already be in the cache (pa_reshape_and_cache
+ * first).  q, out: device fp16 [num_tokens][num_heads][head_dim];
+ * block_tables: device int32 [num_reqs][max_blocks]; ctx_before: device int32
+ * [num_reqs].  Rows of out not covered by any request are left unwritten.
+ * QK^T and PV run on the tcgen05 tensor cores (fp16 operands, fp32 TMEM
+ * accumulators); the softmax runs in fp32.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+pa_status pa_paged_attention_prefill_chunk(pa_half* out, const pa_half* q,
+                                           const pa_half* k_cache, const pa_half* v_cache,
+                                           const int32_t* block_tables, const int32_t* q_start,
+                                           const int32_t* ctx_before, int32_t num_reqs,
+                                           int32_t num_tokens, int32_t num_heads, int32_t head_dim,
+                                           int32_t block_size, int32_t max_blocks,
+                                           int32_t num_blocks, float scale,
+                                           int32_t* err_flag, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PAGEDKV_H */

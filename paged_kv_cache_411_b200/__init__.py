@@ -1,0 +1,194 @@
+"""Paged-KV attention for NVIDIA B200 (sm_100a): the Python face of libpagedkv.so.
+
+The functions and the ``BlockAllocator`` class carry the names of the C entry
+points in ``include/pagedkv.h`` and only marshal arguments: torch tensors are
+used for device memory and streams, every computation runs in the library.
+
+    reshape_and_cache(k_new, v_new, k_cache, v_cache, slot_mapping)
+    paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, scale, workspace)
+    paged_attention_prefill_chunk(out, q, k_cache, v_cache, block_tables, q_start, ctx_before, scale)
+    BlockAllocator(num_blocks, block_size, free_order=None)
+"""
+from __future__ import annotations
+
+import ctypes
+from ctypes import POINTER, byref, c_int32, c_int64, c_void_p
+
+import numpy as np
+
+from ._lib import (PA_DEVCHK_BLOCK_ID, PA_DEVCHK_QUERY_RANGE, PA_DEVCHK_SEQ_LEN, PA_DEVCHK_SLOT,
+                   PA_DEVCHK_TIMEOUT, PA_ERR_CUDA, PA_ERR_DEVICE_CHECK, PA_ERR_EXISTS, PA_ERR_INVALID_ARG,
+                   PA_ERR_NOT_FOUND, PA_ERR_OOM, PA_ERR_UNSUPPORTED, PA_OK, STATUS_NAMES, AllocStats,
+                   PagedKVError, check, last_error, lib)
+
+__all__ = [
+    "BlockAllocator", "reshape_and_cache", "paged_attention_decode", "paged_attention_prefill_chunk",
+    "decode_workspace_bytes", "PagedKVError", "lib", "STATUS_NAMES", "PA_OK", "PA_ERR_INVALID_ARG",
+    "PA_ERR_OOM", "PA_ERR_NOT_FOUND", "PA_ERR_EXISTS", "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA",
+    "PA_ERR_DEVICE_CHECK", "PA_DEVCHK_BLOCK_ID", "PA_DEVCHK_SLOT", "PA_DEVCHK_SEQ_LEN",
+    "PA_DEVCHK_QUERY_RANGE", "PA_DEVCHK_TIMEOUT",
+]
+
+
+def _i32p(a: np.ndarray):
+    return a.ctypes.data_as(POINTER(c_int32))
+
+
+def _i64p(a: np.ndarray):
+    return a.ctypes.data_as(POINTER(c_int64))
+
+
+class BlockAllocator:
+    """Host block allocator (pa_alloc_*).  Methods return the C status code
+    (``PA_OK`` ...) plus their outputs, exactly as the C calls report them."""
+
+    def __init__(self, num_blocks: int, block_size: int, free_order=None):
+        self._h = c_void_p()
+        order = None
+        if free_order is not None:
+            order = np.ascontiguousarray(free_order, dtype=np.int32)
+        check(lib().pa_alloc_create(num_blocks, block_size, None if order is None else _i32p(order),
+                                    byref(self._h)))
+        self.num_blocks = int(num_blocks)
+        self.block_size = int(block_size)
+
+    def close(self):
+        if self._h:
+            lib().pa_alloc_destroy(self._h)
+            self._h = c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def allocate(self, req: int, num_tokens: int) -> int:
+        return lib().pa_alloc_allocate(self._h, req, num_tokens)
+
+    def append_token(self, req: int):
+        slot = c_int64(-1)
+        st = lib().pa_alloc_append_token(self._h, req, byref(slot))
+        return st, (slot.value if st == PA_OK else None)
+
+    def append_tokens(self, req: int, n: int):
+        out = np.empty(max(n, 0), dtype=np.int64)
+        st = lib().pa_alloc_append_tokens(self._h, req, n, _i64p(out))
+        return st, (out if st == PA_OK else np.empty(0, np.int64))
+
+    def fork(self, src: int, dst: int, prefix_tokens: int) -> int:
+        return lib().pa_alloc_fork(self._h, src, dst, prefix_tokens)
+
+    def free(self, req: int) -> int:
+        return lib().pa_alloc_free(self._h, req)
+
+    def get_block_table(self, req: int):
+        n = c_int32(0)
+        st = lib().pa_alloc_get_block_table(self._h, req, None, 0, byref(n))
+        if st == PA_ERR_NOT_FOUND:
+            return st, np.empty(0, np.int32)
+        out = np.empty(n.value, dtype=np.int32)
+        st = lib().pa_alloc_get_block_table(self._h, req, _i32p(out), n.value, byref(n))
+        return st, out
+
+    def seq_len(self, req: int):
+        n = c_int32(0)
+        st = lib().pa_alloc_seq_len(self._h, req, byref(n))
+        return st, (n.value if st == PA_OK else None)
+
+    def slots(self, req: int, pos_begin: int, n: int):
+        out = np.empty(max(n, 0), dtype=np.int64)
+        st = lib().pa_alloc_slots(self._h, req, pos_begin, n, _i64p(out))
+        return st, out
+
+    def pack(self, reqs, max_blocks: int):
+        r = np.ascontiguousarray(reqs, dtype=np.int64)
+        tables = np.empty((len(r), max_blocks), dtype=np.int32)
+        lens = np.empty(len(r), dtype=np.int32)
+        st = lib().pa_alloc_pack(self._h, _i64p(r), len(r), max_blocks, _i32p(tables), _i32p(lens))
+        return st, tables, lens
+
+    def stats(self) -> dict:
+        s = AllocStats()
+        check(lib().pa_alloc_stats(self._h, byref(s)))
+        return s.as_dict()
+
+    def refcount(self, block: int):
+        n = c_int32(0)
+        st = lib().pa_alloc_refcount(self._h, block, byref(n))
+        return st, n.value
+
+    def free_list(self) -> np.ndarray:
+        n = c_int32(0)
+        lib().pa_alloc_free_list(self._h, None, 0, byref(n))
+        out = np.empty(n.value, dtype=np.int32)
+        check(lib().pa_alloc_free_list(self._h, _i32p(out), n.value, byref(n)))
+        return out
+
+
+# ------------------------------------------------------------------ kernels
+def _ptr(t):
+    return None if t is None else c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return c_void_p(stream.cuda_stream)
+
+
+def _need(cond, msg):
+    if not cond:
+        raise PagedKVError(PA_ERR_INVALID_ARG, msg)
+
+
+def reshape_and_cache(k_new, v_new, k_cache, v_cache, slot_mapping, err_flag=None, stream=None):
+    """pa_reshape_and_cache on torch tensors: k_new/v_new [T,H,D] fp16, caches [NB,bs,H,D] fp16,
+    slot_mapping [T] int64 (device)."""
+    import torch
+    _need(k_new.dtype == torch.float16 and k_cache.dtype == torch.float16, "fp16 tensors expected")
+    _need(slot_mapping.dtype == torch.int64, "slot_mapping must be int64")
+    _need(all(t.is_contiguous() for t in (k_new, v_new, k_cache, v_cache, slot_mapping)), "contiguous tensors expected")
+    T, H, D = k_new.shape
+    NB, bs = k_cache.shape[:2]
+    check(lib().pa_reshape_and_cache(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping),
+                                     T, H, D, bs, NB, _ptr(err_flag), _stream(stream)))
+
+
+def decode_workspace_bytes(num_seqs: int, num_heads: int, head_dim: int, max_blocks: int, block_size: int) -> int:
+    return int(lib().pa_decode_workspace_bytes(num_seqs, num_heads, head_dim, max_blocks, block_size))
+
+
+def paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, scale, workspace,
+                           err_flag=None, stream=None):
+    """pa_paged_attention_decode on torch tensors: out/q [S,H,D] fp16, caches [NB,bs,H,D] fp16,
+    block_tables [S,max_blocks] int32, seq_lens [S] int32, workspace uint8 (device)."""
+    import torch
+    _need(q.dtype == torch.float16 and out.dtype == torch.float16, "fp16 tensors expected")
+    _need(block_tables.dtype == torch.int32 and seq_lens.dtype == torch.int32, "int32 tables expected")
+    _need(all(t.is_contiguous() for t in (out, q, k_cache, v_cache, block_tables, seq_lens)), "contiguous tensors expected")
+    S, H, D = q.shape
+    NB, bs = k_cache.shape[:2]
+    max_blocks = block_tables.shape[1] if block_tables.dim() == 2 else 0
+    check(lib().pa_paged_attention_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                                          _ptr(seq_lens), S, H, D, bs, max_blocks, NB, float(scale),
+                                          _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                          _ptr(err_flag), _stream(stream)))
+
+
+def paged_attention_prefill_chunk(out, q, k_cache, v_cache, block_tables, q_start, ctx_before, scale,
+                                  err_flag=None, stream=None):
+    """pa_paged_attention_prefill_chunk on torch tensors: out/q [T,H,D] fp16, caches [NB,bs,H,D] fp16,
+    block_tables [B,max_blocks] int32, q_start [B+1] int32, ctx_before [B] int32 (device)."""
+    import torch
+    _need(q.dtype == torch.float16 and out.dtype == torch.float16, "fp16 tensors expected")
+    _need(all(t.is_contiguous() for t in (out, q, k_cache, v_cache, block_tables, q_start, ctx_before)),
+          "contiguous tensors expected")
+    T, H, D = q.shape
+    NB, bs = k_cache.shape[:2]
+    B = ctx_before.shape[0]
+    check(lib().pa_paged_attention_prefill_chunk(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                                 _ptr(block_tables), _ptr(q_start), _ptr(ctx_before), B, T, H, D,
+                                                 bs, block_tables.shape[1], NB, float(scale), _ptr(err_flag),
+                                                 _stream(stream)))

@@ -1,0 +1,273 @@
+// Host block allocator of libpagedkv.
+//
+// The pool, free list and per-request block tables of the block manager on
+// the page "LLM 推理引擎 Continuous Batching 与 PagedAttention" (§3.2 核心数据
+// 结构), with the refcounted shared-prefix blocks of §4.1.  Semantics:
+//   * the free list is a stack: every take pops its end; blocks whose refcount
+//     reaches zero are pushed on the end in block-table order;
+//   * allocate / append_tokens are all-or-nothing; OOM leaves every field as
+//     it was and bumps oom_count;
+//   * append_token takes a block iff the request's current length is a
+//     multiple of block_size (current length = tokens stored before the call);
+//   * fork shares whole blocks only (floor(prefix / block_size));
+//   * a token's slot is table[pos / block_size] * block_size + pos % block_size
+//     (the address form of the page's §3.3 kernel).
+// Everything is O(1) per token except free, which is O(table length).
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <unordered_map>
+#include <vector>
+
+#include "common.h"
+
+namespace pagedkv {
+
+static thread_local std::string g_last_error;
+
+pa_status fail(pa_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+void clear_error() { g_last_error.clear(); }
+
+const char* last_error() { return g_last_error.c_str(); }
+
+}  // namespace pagedkv
+
+using pagedkv::fail;
+
+struct pa_alloc {
+    struct Request {
+        std::vector<int32_t> table;
+        int32_t len = 0;
+    };
+    int32_t num_blocks = 0;
+    int32_t block_size = 0;
+    std::vector<int32_t> free_list;      // stack; back() is the next pop
+    std::vector<int32_t> refcount;
+    std::unordered_map<int64_t, Request> reqs;
+    int64_t oom_count = 0;
+
+    int64_t blocks_for(int64_t tokens) const { return (tokens + block_size - 1) / block_size; }
+    int32_t take() {
+        int32_t b = free_list.back();
+        free_list.pop_back();
+        refcount[b] += 1;
+        return b;
+    }
+    int64_t slot(const Request& r, int64_t pos) const {
+        return static_cast<int64_t>(r.table[pos / block_size]) * block_size + pos % block_size;
+    }
+};
+
+extern "C" {
+
+pa_status pa_alloc_create(int32_t num_blocks, int32_t block_size, const int32_t* init_free_order,
+                          pa_alloc** out) {
+    if (!out) return fail(PA_ERR_INVALID_ARG, "pa_alloc_create: out is NULL");
+    *out = nullptr;
+    if (num_blocks < 0 || block_size <= 0)
+        return fail(PA_ERR_INVALID_ARG, "pa_alloc_create: num_blocks=%d block_size=%d", num_blocks, block_size);
+    pa_alloc* a = new (std::nothrow) pa_alloc();
+    if (!a) return fail(PA_ERR_OOM, "pa_alloc_create: host allocation failed");
+    a->num_blocks = num_blocks;
+    a->block_size = block_size;
+    a->refcount.assign(num_blocks, 0);
+    a->free_list.resize(num_blocks);
+    if (init_free_order) {
+        std::vector<char> seen(num_blocks, 0);
+        for (int32_t i = 0; i < num_blocks; ++i) {
+            int32_t b = init_free_order[i];
+            if (b < 0 || b >= num_blocks || seen[b]) {
+                delete a;
+                return fail(PA_ERR_INVALID_ARG, "pa_alloc_create: init_free_order is not a permutation (entry %d = %d)", i, b);
+            }
+            seen[b] = 1;
+            a->free_list[i] = b;
+        }
+    } else {
+        for (int32_t i = 0; i < num_blocks; ++i) a->free_list[i] = i;
+    }
+    *out = a;
+    return PA_OK;
+}
+
+void pa_alloc_destroy(pa_alloc* a) { delete a; }
+
+pa_status pa_alloc_allocate(pa_alloc* a, int64_t req, int32_t num_tokens) {
+    if (!a) return fail(PA_ERR_INVALID_ARG, "pa_alloc_allocate: NULL allocator");
+    if (num_tokens < 0) return fail(PA_ERR_INVALID_ARG, "pa_alloc_allocate: num_tokens=%d", num_tokens);
+    if (a->reqs.count(req)) return fail(PA_ERR_EXISTS, "pa_alloc_allocate: request %lld exists", (long long)req);
+    int64_t n = a->blocks_for(num_tokens);
+    if (n > static_cast<int64_t>(a->free_list.size())) {
+        a->oom_count += 1;
+        return fail(PA_ERR_OOM, "pa_alloc_allocate: need %lld blocks, %zu free", (long long)n, a->free_list.size());
+    }
+    pa_alloc::Request r;
+    r.table.reserve(n);
+    for (int64_t i = 0; i < n; ++i) r.table.push_back(a->take());
+    r.len = num_tokens;
+    a->reqs.emplace(req, std::move(r));
+    return PA_OK;
+}
+
+pa_status pa_alloc_append_token(pa_alloc* a, int64_t req, int64_t* slot_out) {
+    if (!a) return fail(PA_ERR_INVALID_ARG, "pa_alloc_append_token: NULL allocator");
+    auto it = a->reqs.find(req);
+    if (it == a->reqs.end()) return fail(PA_ERR_NOT_FOUND, "pa_alloc_append_token: request %lld not found", (long long)req);
+    pa_alloc::Request& r = it->second;
+    if (r.len % a->block_size == 0) {
+        if (a->free_list.empty()) {
+            a->oom_count += 1;
+            return fail(PA_ERR_OOM, "pa_alloc_append_token: no free block");
+        }
+        r.table.push_back(a->take());
+    }
+    if (slot_out) *slot_out = a->slot(r, r.len);
+    r.len += 1;
+    return PA_OK;
+}
+
+pa_status pa_alloc_append_tokens(pa_alloc* a, int64_t req, int32_t n, int64_t* slots_out) {
+    if (!a) return fail(PA_ERR_INVALID_ARG, "pa_alloc_append_tokens: NULL allocator");
+    if (n < 0) return fail(PA_ERR_INVALID_ARG, "pa_alloc_append_tokens: n=%d", n);
+    auto it = a->reqs.find(req);
+    if (it == a->reqs.end()) return fail(PA_ERR_NOT_FOUND, "pa_alloc_append_tokens: request %lld not found", (long long)req);
+    pa_alloc::Request& r = it->second;
+    int64_t extra = a->blocks_for(static_cast<int64_t>(r.len) + n) - static_cast<int64_t>(r.table.size());
+    if (extra > static_cast<int64_t>(a->free_list.size())) {
+        a->oom_count += 1;
+        return fail(PA_ERR_OOM, "pa_alloc_append_tokens: need %lld blocks, %zu free", (long long)extra, a->free_list.size());
+    }
+    for (int32_t i = 0; i < n; ++i) {
+        if (r.len % a->block_size == 0) r.table.push_back(a->take());
+        if (slots_out) slots_out[i] = a->slot(r, r.len);
+        r.len += 1;
+    }
+    return PA_OK;
+}
+
+pa_status pa_alloc_fork(pa_alloc* a, int64_t src, int64_t dst, int32_t prefix_tokens) {
+    if (!a) return fail(PA_ERR_INVALID_ARG, "pa_alloc_fork: NULL allocator");
+    auto it = a->reqs.find(src);
+    if (it == a->reqs.end()) return fail(PA_ERR_NOT_FOUND, "pa_alloc_fork: source %lld not found", (long long)src);
+    if (a->reqs.count(dst)) return fail(PA_ERR_EXISTS, "pa_alloc_fork: destination %lld exists", (long long)dst);
+    if (prefix_tokens < 0 || prefix_tokens > it->second.len)
+        return fail(PA_ERR_INVALID_ARG, "pa_alloc_fork: prefix_tokens=%d, source holds %d", prefix_tokens, it->second.len);
+    int32_t shared = prefix_tokens / a->block_size;
+    pa_alloc::Request r;
+    r.table.assign(it->second.table.begin(), it->second.table.begin() + shared);
+    for (int32_t b : r.table) a->refcount[b] += 1;
+    r.len = shared * a->block_size;
+    a->reqs.emplace(dst, std::move(r));
+    return PA_OK;
+}
+
+pa_status pa_alloc_free(pa_alloc* a, int64_t req) {
+    if (!a) return fail(PA_ERR_INVALID_ARG, "pa_alloc_free: NULL allocator");
+    auto it = a->reqs.find(req);
+    if (it == a->reqs.end()) return PA_OK;
+    for (int32_t b : it->second.table) {
+        if (--a->refcount[b] == 0) a->free_list.push_back(b);
+    }
+    a->reqs.erase(it);
+    return PA_OK;
+}
+
+pa_status pa_alloc_get_block_table(const pa_alloc* a, int64_t req, int32_t* out, int32_t cap, int32_t* len_out) {
+    if (!a) return fail(PA_ERR_INVALID_ARG, "pa_alloc_get_block_table: NULL allocator");
+    auto it = a->reqs.find(req);
+    if (it == a->reqs.end()) return fail(PA_ERR_NOT_FOUND, "pa_alloc_get_block_table: request %lld not found", (long long)req);
+    int32_t n = static_cast<int32_t>(it->second.table.size());
+    if (len_out) *len_out = n;
+    if (cap < n || (n > 0 && !out))
+        return fail(PA_ERR_INVALID_ARG, "pa_alloc_get_block_table: capacity %d < table length %d", cap, n);
+    if (n) std::memcpy(out, it->second.table.data(), sizeof(int32_t) * n);
+    return PA_OK;
+}
+
+pa_status pa_alloc_seq_len(const pa_alloc* a, int64_t req, int32_t* out) {
+    if (!a || !out) return fail(PA_ERR_INVALID_ARG, "pa_alloc_seq_len: NULL argument");
+    auto it = a->reqs.find(req);
+    if (it == a->reqs.end()) return fail(PA_ERR_NOT_FOUND, "pa_alloc_seq_len: request %lld not found", (long long)req);
+    *out = it->second.len;
+    return PA_OK;
+}
+
+pa_status pa_alloc_slots(const pa_alloc* a, int64_t req, int32_t pos_begin, int32_t n, int64_t* slots_out) {
+    if (!a) return fail(PA_ERR_INVALID_ARG, "pa_alloc_slots: NULL allocator");
+    auto it = a->reqs.find(req);
+    if (it == a->reqs.end()) return fail(PA_ERR_NOT_FOUND, "pa_alloc_slots: request %lld not found", (long long)req);
+    const pa_alloc::Request& r = it->second;
+    if (pos_begin < 0 || n < 0 || static_cast<int64_t>(pos_begin) + n > r.len || (n > 0 && !slots_out))
+        return fail(PA_ERR_INVALID_ARG, "pa_alloc_slots: positions [%d, %d) outside [0, %d)", pos_begin, pos_begin + n, r.len);
+    for (int32_t i = 0; i < n; ++i) slots_out[i] = a->slot(r, static_cast<int64_t>(pos_begin) + i);
+    return PA_OK;
+}
+
+pa_status pa_alloc_pack(const pa_alloc* a, const int64_t* reqs, int32_t n, int32_t max_blocks,
+                        int32_t* tables, int32_t* seq_lens) {
+    if (!a || n < 0 || max_blocks < 0 || (n > 0 && (!reqs || !tables || !seq_lens)))
+        return fail(PA_ERR_INVALID_ARG, "pa_alloc_pack: bad arguments");
+    std::vector<const pa_alloc::Request*> rs(n);
+    for (int32_t i = 0; i < n; ++i) {
+        auto it = a->reqs.find(reqs[i]);
+        if (it == a->reqs.end()) return fail(PA_ERR_NOT_FOUND, "pa_alloc_pack: request %lld not found", (long long)reqs[i]);
+        if (static_cast<int64_t>(it->second.table.size()) > max_blocks)
+            return fail(PA_ERR_INVALID_ARG, "pa_alloc_pack: request %lld holds %zu blocks > max_blocks %d",
+                        (long long)reqs[i], it->second.table.size(), max_blocks);
+        rs[i] = &it->second;
+    }
+    for (int32_t i = 0; i < n; ++i) {
+        int32_t* row = tables + static_cast<int64_t>(i) * max_blocks;
+        size_t k = rs[i]->table.size();
+        if (k) std::memcpy(row, rs[i]->table.data(), sizeof(int32_t) * k);
+        for (int32_t j = static_cast<int32_t>(k); j < max_blocks; ++j) row[j] = -1;
+        seq_lens[i] = rs[i]->len;
+    }
+    return PA_OK;
+}
+
+pa_status pa_alloc_stats(const pa_alloc* a, pa_alloc_stats_t* out) {
+    if (!a || !out) return fail(PA_ERR_INVALID_ARG, "pa_alloc_stats: NULL argument");
+    pa_alloc_stats_t s{};
+    s.num_blocks = a->num_blocks;
+    s.block_size = a->block_size;
+    s.num_free = static_cast<int32_t>(a->free_list.size());
+    for (int32_t c : a->refcount) {
+        if (c > 0) s.num_used += 1;
+        s.total_refs += c;
+    }
+    s.num_requests = static_cast<int64_t>(a->reqs.size());
+    s.oom_count = a->oom_count;
+    for (const auto& kv : a->reqs)
+        s.waste_tokens += static_cast<int64_t>(kv.second.table.size()) * a->block_size - kv.second.len;
+    *out = s;
+    return PA_OK;
+}
+
+pa_status pa_alloc_refcount(const pa_alloc* a, int32_t block, int32_t* out) {
+    if (!a || !out || block < 0 || block >= a->num_blocks)
+        return fail(PA_ERR_INVALID_ARG, "pa_alloc_refcount: bad block %d", block);
+    *out = a->refcount[block];
+    return PA_OK;
+}
+
+pa_status pa_alloc_free_list(const pa_alloc* a, int32_t* out, int32_t cap, int32_t* len_out) {
+    if (!a) return fail(PA_ERR_INVALID_ARG, "pa_alloc_free_list: NULL allocator");
+    int32_t n = static_cast<int32_t>(a->free_list.size());
+    if (len_out) *len_out = n;
+    if (cap < n || (n > 0 && !out)) return fail(PA_ERR_INVALID_ARG, "pa_alloc_free_list: capacity %d < %d", cap, n);
+    if (n) std::memcpy(out, a->free_list.data(), sizeof(int32_t) * n);
+    return PA_OK;
+}
+
+}  // extern "C"
