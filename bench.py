@@ -328,7 +328,7 @@ def run_ours(args):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="b256", choices=sorted(si.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
