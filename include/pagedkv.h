@@ -222,6 +222,28 @@ pa_status pa_paged_attention_decode(pa_half* out, const pa_half* q,
                                     float scale, void* workspace, size_t workspace_bytes,
                                     int32_t* err_flag, void* stream);
 
+/* pa_paged_attention_decode for callers that cannot allocate device memory.
+ * The pages describe no counterpart of this entry point; it exists for code
+ * that is handed fixed buffers and may not call cudaMalloc (allocator-less
+ * embedded loops, plugins whose host forbids allocation after start-up,
+ * latency-critical paths that must avoid cudaMalloc's implicit
+ * synchronisation).  Same arguments and results as pa_paged_attention_decode
+ * minus the workspace: the scratch comes from a fixed 64 MiB (67108864-byte)
+ * array that the library keeps in device memory on every GPU that loads it,
+ * until the process exits.  A batch whose pa_decode_workspace_bytes exceeds
+ * that returns PA_ERR_INVALID_ARG with a message saying so.  The first call on
+ * a device looks the array's address up (cudaGetSymbolAddress, with that
+ * device current); make that first call before any stream capture.  Calls on
+ * one device share the array: calls whose kernels may overlap on the GPU race
+ * and must be serialised by the caller.  Allocates nothing.
+ * Errors: as pa_paged_attention_decode. */
+pa_status pa_paged_attention_decode_noalloc(pa_half* out, const pa_half* q,
+                                            const pa_half* k_cache, const pa_half* v_cache,
+                                            const int32_t* block_tables, const int32_t* seq_lens,
+                                            int32_t num_seqs, int32_t num_heads, int32_t head_dim,
+                                            int32_t block_size, int32_t max_blocks, int32_t num_blocks,
+                                            float scale, int32_t* err_flag, void* stream);
+
 /* Chunked-prefill attention over the paged cache ([CB-PA] §4.3 Chunked
  * Prefill; §1.1 prefill phase).  Request b < num_reqs owns query rows
  * q_start[b] .. q_start[b+1]-1 (host-unknown, device int32 [num_reqs+1],

@@ -23,7 +23,7 @@ from ._lib import (PA_DEVCHK_BLOCK_ID, PA_DEVCHK_QUERY_RANGE, PA_DEVCHK_SEQ_LEN,
 
 __all__ = [
     "BlockAllocator", "reshape_and_cache", "paged_attention_decode", "paged_attention_prefill_chunk",
-    "decode_workspace_bytes", "PagedKVError", "lib", "STATUS_NAMES", "PA_OK", "PA_ERR_INVALID_ARG",
+    "decode_workspace_bytes", "paged_attention_decode_noalloc", "PagedKVError", "lib", "STATUS_NAMES", "PA_OK", "PA_ERR_INVALID_ARG",
     "PA_ERR_OOM", "PA_ERR_NOT_FOUND", "PA_ERR_EXISTS", "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA",
     "PA_ERR_DEVICE_CHECK", "PA_DEVCHK_BLOCK_ID", "PA_DEVCHK_SLOT", "PA_DEVCHK_SEQ_LEN",
     "PA_DEVCHK_QUERY_RANGE", "PA_DEVCHK_TIMEOUT",
@@ -175,6 +175,22 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, sca
                                           _ptr(seq_lens), S, H, D, bs, max_blocks, NB, float(scale),
                                           _ptr(workspace), workspace.numel() * workspace.element_size(),
                                           _ptr(err_flag), _stream(stream)))
+
+
+def paged_attention_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, scale, err_flag=None,
+                                   stream=None):
+    """pa_paged_attention_decode_noalloc on torch tensors: as paged_attention_decode, with the
+    library's fixed device scratch instead of a caller workspace (for callers that cannot allocate)."""
+    import torch
+    _need(q.dtype == torch.float16 and out.dtype == torch.float16, "fp16 tensors expected")
+    _need(block_tables.dtype == torch.int32 and seq_lens.dtype == torch.int32, "int32 tables expected")
+    _need(all(t.is_contiguous() for t in (out, q, k_cache, v_cache, block_tables, seq_lens)), "contiguous tensors expected")
+    S, H, D = q.shape
+    NB, bs = k_cache.shape[:2]
+    check(lib().pa_paged_attention_decode_noalloc(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                                  _ptr(block_tables), _ptr(seq_lens), S, H, D, bs,
+                                                  block_tables.shape[1], NB, float(scale), _ptr(err_flag),
+                                                  _stream(stream)))
 
 
 def paged_attention_prefill_chunk(out, q, k_cache, v_cache, block_tables, q_start, ctx_before, scale,

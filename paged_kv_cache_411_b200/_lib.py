@@ -80,6 +80,8 @@ SIGNATURES = {
     "pa_decode_workspace_bytes": (c_size_t, [c_int32, c_int32, c_int32, c_int32, c_int32]),
     "pa_paged_attention_decode": (c_int32, [_P, _P, _P, _P, _P, _P, c_int32, c_int32, c_int32, c_int32, c_int32,
                                             c_int32, c_float, _P, c_size_t, _P, _P]),
+    "pa_paged_attention_decode_noalloc": (c_int32, [_P, _P, _P, _P, _P, _P, c_int32, c_int32, c_int32, c_int32,
+                                                    c_int32, c_int32, c_float, _P, _P]),
     "pa_paged_attention_prefill_chunk": (c_int32, [_P, _P, _P, _P, _P, _P, _P, c_int32, c_int32, c_int32, c_int32,
                                                    c_int32, c_int32, c_int32, c_float, _P, _P]),
 }

@@ -29,6 +29,7 @@ SOURCES = [
     "runtime.cpp",
     "reshape_and_cache.cu",
     "decode.cu",
+    "decode_noalloc.cu",
     "prefill.cu",
 ]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
