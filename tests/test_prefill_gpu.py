@@ -1,0 +1,154 @@
+"""GPU parity of the tcgen05 chunked-prefill kernel against the CPU oracle.
+
+Max abs error <= 2e-3 against the float64 oracle (fp16 operands, fp32 TMEM
+accumulation, P rounded to fp16 for the second MMA, fp16 output)."""
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_411_b200 as pk
+import synth_inputs as si
+from oracle import attention as oatt
+from oracle import workloads as owl
+from paged_kv_cache_411_b200 import workload as pwl
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-3
+
+
+def make_case(seed, H, D, bs, reqs, extra_blocks=5, garbage_pad=True):
+    """reqs: [(ctx_before, chunk_len)].  The pool holds every request's ctx + chunk rows at
+    shuffled blocks; unused rows are NaN.  Returns numpy and device views."""
+    rng = np.random.default_rng(seed)
+    need = [-(-(c + L) // bs) for c, L in reqs]
+    N = sum(need) + extra_blocks
+    order = rng.permutation(N)
+    kc = np.full((N, bs, H, D), np.nan, np.float16)
+    vc = np.full((N, bs, H, D), np.nan, np.float16)
+    maxb = max(need + [1]) + 2
+    tables = rng.integers(0, N, size=(len(reqs), maxb)).astype(np.int32) if garbage_pad else \
+        np.full((len(reqs), maxb), -1, np.int32)
+    nxt = 0
+    for b, (c, L) in enumerate(reqs):
+        t = order[nxt:nxt + need[b]]
+        nxt += need[b]
+        tables[b, :len(t)] = t
+        n = c + L
+        k = rng.standard_normal((n, H, D)).astype(np.float16)
+        v = rng.standard_normal((n, H, D)).astype(np.float16)
+        for j in range(n):
+            kc[t[j // bs], j % bs] = k[j]
+            vc[t[j // bs], j % bs] = v[j]
+    T = sum(L for _, L in reqs)
+    q = rng.standard_normal((T, H, D)).astype(np.float16)
+    q_start = np.concatenate([[0], np.cumsum([L for _, L in reqs])]).astype(np.int32)
+    ctx = np.asarray([c for c, _ in reqs], np.int32)
+    dev = {k_: torch.from_numpy(v_).cuda() for k_, v_ in
+           dict(q=q, kc=kc, vc=vc, tables=tables, q_start=q_start, ctx=ctx).items()}
+    return dict(q=q, kc=kc, vc=vc, tables=tables, q_start=q_start, ctx=ctx, dev=dev)
+
+
+def run_prefill(case, scale, err=None):
+    d = case["dev"]
+    out = torch.full_like(d["q"], float("nan"))
+    pk.paged_attention_prefill_chunk(out, d["q"], d["kc"], d["vc"], d["tables"], d["q_start"], d["ctx"], scale,
+                                     err_flag=err)
+    return out
+
+
+def oracle_prefill(case, bs, scale):
+    return oatt.paged_attention_prefill_chunk(case["q"], case["kc"], case["vc"], case["tables"],
+                                              case["q_start"], case["ctx"], bs, scale)
+
+
+CASES = [
+    # (H, D, bs, [(ctx_before, chunk)])
+    (2, 128, 16, [(0, 128)]),
+    (2, 128, 16, [(0, 70)]),
+    (2, 128, 16, [(1536, 512)]),
+    (4, 128, 16, [(37, 200)]),
+    (3, 64, 16, [(0, 300)]),
+    (2, 64, 32, [(100, 129)]),
+    (2, 128, 8, [(55, 90)]),
+    (2, 128, 64, [(130, 260)]),
+    (2, 128, 48, [(47, 81)]),
+    (4, 128, 16, [(0, 1), (300, 40), (17, 256), (5, 0), (1000, 130)]),
+    (8, 64, 16, [(64, 64), (0, 2), (129, 383)]),
+]
+
+
+@pytest.mark.parametrize("H,D,bs,reqs", CASES)
+def test_prefill_matches_oracle(cuda_ready, H, D, bs, reqs):
+    case = make_case(hash((H, D, bs, len(reqs))) % 1000, H, D, bs, reqs)
+    scale = 1 / np.sqrt(D)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = run_prefill(case, scale, err).float().cpu().numpy()
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    ref = oracle_prefill(case, bs, scale)
+    assert np.isfinite(out).all()
+    diff = np.abs(out - ref)
+    assert diff.max() <= TOL, f"max abs error {diff.max():.3g}"
+
+
+def test_mixed_workload_prefill(cuda_ready):
+    """The 512-row chunk after 1536 cached tokens of the mixed step, 32 heads x 128."""
+    w = si.get("mixed")
+    ds = pwl.build(w)
+    pk.reshape_and_cache(ds.k_step, ds.v_step, ds.k_cache, ds.v_cache, ds.slot_mapping)
+    out = torch.empty_like(ds.prefill_q)
+    pk.paged_attention_prefill_chunk(out, ds.prefill_q, ds.k_cache, ds.v_cache, ds.prefill_table,
+                                     ds.prefill_q_start, ds.prefill_ctx_before, w.scale)
+    got = out.float().cpu().numpy()
+    o = owl.build(w, seqs=[0])
+    _, pre, _, _ = owl.run_step(o)
+    diff = np.abs(got - pre)
+    assert diff.max() <= TOL, f"max abs error {diff.max():.3g}"
+
+
+def test_chunk_split_and_decode_agree(cuda_ready):
+    """Chunking is a scheduling split: two chunks give the rows one chunk gives, and the last
+    row equals the decode kernel's output at the same context (within the tolerance)."""
+    H, D, bs, c, L = 4, 128, 16, 300, 200
+    case = make_case(3, H, D, bs, [(c, L)])
+    scale = 1 / np.sqrt(D)
+    whole = run_prefill(case, scale).float()
+    d = case["dev"]
+    parts = []
+    for lo, hi in ((0, 77), (77, L)):
+        out = torch.empty(hi - lo, H, D, dtype=torch.float16, device="cuda")
+        pk.paged_attention_prefill_chunk(out, d["q"][lo:hi].contiguous(), d["kc"], d["vc"], d["tables"],
+                                         torch.tensor([0, hi - lo], dtype=torch.int32, device="cuda"),
+                                         torch.tensor([c + lo], dtype=torch.int32, device="cuda"), scale)
+        parts.append(out.float())
+    assert (whole - torch.cat(parts)).abs().max().item() <= TOL
+    ws = torch.empty(pk.decode_workspace_bytes(1, H, D, d["tables"].shape[1], bs), dtype=torch.uint8, device="cuda")
+    dec = torch.empty(1, H, D, dtype=torch.float16, device="cuda")
+    pk.paged_attention_decode(dec, d["q"][L - 1:L].contiguous(), d["kc"], d["vc"], d["tables"],
+                              torch.tensor([c + L], dtype=torch.int32, device="cuda"), scale, ws)
+    assert (whole[L - 1] - dec[0].float()).abs().max().item() <= TOL
+
+
+def test_prefill_device_checks(cuda_ready):
+    case = make_case(4, 2, 128, 16, [(20, 40)])
+    d = case["dev"]
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.zeros_like(d["q"])
+    bad_start = torch.tensor([0, 41], dtype=torch.int32, device="cuda")     # past num_tokens
+    pk.paged_attention_prefill_chunk(out, d["q"], d["kc"], d["vc"], d["tables"], bad_start, d["ctx"], 0.1,
+                                     err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & pk.PA_DEVCHK_QUERY_RANGE
+    err.zero_()
+    tables = d["tables"].clone()
+    tables[0, 1] = 10_000
+    pk.paged_attention_prefill_chunk(out, d["q"], d["kc"], d["vc"], tables, d["q_start"], d["ctx"], 0.1,
+                                     err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == pk.PA_DEVCHK_BLOCK_ID
+    err.zero_()
+    big_ctx = torch.tensor([10_000], dtype=torch.int32, device="cuda")
+    pk.paged_attention_prefill_chunk(out, d["q"], d["kc"], d["vc"], d["tables"], d["q_start"], big_ctx, 0.1,
+                                     err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & pk.PA_DEVCHK_SEQ_LEN
