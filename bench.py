@@ -37,13 +37,26 @@ METRIC = "paged-attn decode GB/s (% of B200 HBM peak) and decode tokens/s at 1 G
 FALLBACK_HBM_GBS = 6650.0
 
 
+FALLBACK_TFLOPS = 1590.0
+
+
 def measured_peaks():
+    """(HBM GB/s, dense fp16/bf16 tensor TFLOP/s burst, kind)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
-    return FALLBACK_HBM_GBS, "fallback"
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_TFLOPS, "fallback"
+
+
+def prefill_flops(w):
+    """Algorithmic FLOPs of the causal chunk: 4 * H * D per visible (query, key) pair."""
+    if w.prefill is None:
+        return 0
+    L, c = w.prefill.chunk, w.prefill.ctx_before
+    pairs = L * c + L * (L + 1) // 2
+    return 4 * w.num_heads * w.head_dim * pairs
 
 
 def step_bytes(w, seq_lens, tables_cols, n_step_rows):
@@ -146,8 +159,7 @@ def oracle_sample_seqs(w, budget_tokens):
     return sorted(pick)
 
 
-def time_oracle(w, steps, warmup, budget_tokens):
-    """Times the CPU oracle's decode on a bounded sample; returns (GB/s, s/step, sample desc, threads)."""
+def _oracle_case(w, budget_tokens):
     from oracle import attention as oatt
     from oracle import workloads as owl
     sample = oracle_sample_seqs(w, budget_tokens)
@@ -156,17 +168,44 @@ def time_oracle(w, steps, warmup, budget_tokens):
     oatt.reshape_and_cache(kc, vc, o.k_step, o.v_step, o.slot_mapping, w.block_size)
     idx = np.asarray(sample)
     args = (o.q[idx], kc, vc, o.block_tables[idx], o.seq_lens[idx], w.block_size, w.scale)
+    tokens = int(o.seq_lens[idx].astype(np.int64).sum())
+    return sample, args, tokens
+
+
+def time_oracle(w, steps, warmup, budget_tokens, min_seconds=0.0, max_steps=None):
+    """Times the CPU oracle's decode on a bounded sample of the workload's sequences.
+
+    Runs ``warmup`` untimed calls, then ``steps`` timed ones (or, with min_seconds, as many as
+    fit in min_seconds up to max_steps).  Returns (GB/s, seconds per step, description, threads)."""
+    from oracle import attention as oatt
+    sample, args, tokens = _oracle_case(w, budget_tokens)
     for _ in range(warmup):
         oatt.paged_attention_decode(*args)
+    n = 0
     t0 = time.perf_counter()
-    for _ in range(steps):
+    while True:
         oatt.paged_attention_decode(*args)
-    dt = (time.perf_counter() - t0) / steps
-    nbytes = int(o.seq_lens[idx].astype(np.int64).sum()) * w.num_heads * w.head_dim * 4
-    threads = _blas_threads()
-    desc = (f"oracle float64 decode of {len(sample)} of {w.num_seqs} sequences "
-            f"({int(o.seq_lens[idx].sum())} cached tokens), GB/s scaled by their K/V bytes")
-    return nbytes / dt / 1e9, dt, desc, threads
+        n += 1
+        el = time.perf_counter() - t0
+        if n >= steps and el >= min_seconds:
+            break
+        if max_steps is not None and n >= max_steps:
+            break
+    dt = el / n
+    nbytes = tokens * w.num_heads * w.head_dim * 4
+    desc = (f"oracle float64 decode of {len(sample)} of {w.num_seqs} sequences ({tokens} cached tokens) per "
+            f"step, {n} timed steps; GB/s counts those sequences' K/V bytes")
+    return nbytes / dt / 1e9, dt, desc, _blas_threads()
+
+
+def oracle_tokens_for(w, total_steps, target_seconds):
+    """Tokens per oracle step so that total_steps steps take about target_seconds on this host."""
+    from oracle import attention as oatt
+    _, args, tokens = _oracle_case(w, 2000)
+    t0 = time.perf_counter()
+    oatt.paged_attention_decode(*args)
+    rate = tokens / max(time.perf_counter() - t0, 1e-6)
+    return int(max(64, min(sum(w.decode_lens), rate * target_seconds / max(1, total_steps))))
 
 
 def _blas_threads():
@@ -183,7 +222,8 @@ def run_reference(args):
     if rank != 0:
         return 0
     w = si.get(args.workload)
-    gbs, dt, desc, threads = time_oracle(w, args.steps, args.warmup, args.oracle_tokens)
+    per_step = oracle_tokens_for(w, args.steps + args.warmup, 120.0)
+    gbs, dt, desc, threads = time_oracle(w, args.steps, args.warmup, per_step)
     line = {
         "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": 0,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
@@ -224,11 +264,15 @@ def run_ours(args):
     dec_b, rs_b, pre_b = step_bytes(w, ds.seq_lens_host, ds.max_blocks, T)
     step_b = dec_b + rs_b + pre_b
 
-    def step(ev=None):
+    def step(ev=None, pev=None):
         pk.reshape_and_cache(ds.k_step, ds.v_step, ds.k_cache, ds.v_cache, ds.slot_mapping, stream=stream)
         if pout is not None:
+            if pev is not None:
+                pev[0].record(stream)
             pk.paged_attention_prefill_chunk(pout, ds.prefill_q, ds.k_cache, ds.v_cache, ds.prefill_table,
                                              ds.prefill_q_start, ds.prefill_ctx_before, w.scale, stream=stream)
+            if pev is not None:
+                pev[1].record(stream)
         if ev is not None:
             ev[0].record(stream)
         pk.paged_attention_decode(out, ds.q, ds.k_cache, ds.v_cache, ds.block_tables, ds.seq_lens, w.scale, ws,
@@ -242,6 +286,8 @@ def run_ours(args):
 
     dec_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                   for _ in range(args.steps)]
+    pre_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)] if pout is not None else [None] * args.steps
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         time.sleep(0.25)
@@ -250,17 +296,18 @@ def run_ours(args):
         torch.cuda.synchronize(device)
         t0.record(stream)
         for i in range(args.steps):
-            step(dec_events[i])
+            step(dec_events[i], pre_events[i])
         t1.record(stream)
         torch.cuda.synchronize(device)
         if world > 1:
             dist.barrier()
     local_ms = t0.elapsed_time(t1)
     dec_ms = [a.elapsed_time(b) for a, b in dec_events]
+    pre_ms = [e[0].elapsed_time(e[1]) for e in pre_events] if pout is not None else []
     total_ms, total_bytes = reduce_max_sum(local_ms, step_b * args.steps, device)
     ms_per_step = total_ms / args.steps
     value = total_bytes / (total_ms / 1e3) / 1e9
-    peak, peak_kind = measured_peaks()
+    peak, peak_tf, peak_kind = measured_peaks()
 
     # end to end: pinned host inputs -> device, the step, the output back to the host, every step
     host = {k: getattr(ds, k).cpu().pin_memory() for k in ("q", "k_step", "v_step", "slot_mapping",
@@ -314,8 +361,16 @@ def run_ours(args):
             "gpu_launches": args.steps * (4 + (1 if pout is not None else 0)),
             "clocks": clk.summary(),
         }
+        if pout is not None:
+            pre_avg = float(np.mean(pre_ms))
+            tf = prefill_flops(w) / (pre_avg / 1e3) / 1e12
+            line["roofline_prefill"] = {
+                "kernel": "paged_attention_prefill_chunk (tcgen05)", "bound": "tensor", "achieved": round(tf, 2),
+                "peak": peak_tf, "peak_kind": peak_kind + " bf16 burst (fp16 has the same nominal rate)",
+                "unit": "TFLOP/s", "frac": round(tf / peak_tf, 4), "traffic": None,
+                "algorithmic_flops_per_launch": prefill_flops(w), "avg_launch_ms": round(pre_avg, 5)}
         if world == 1 and not args.no_cpu_baseline:
-            gbs, dt, desc, threads = time_oracle(w, 1, 0, args.oracle_tokens)
+            gbs, dt, desc, threads = time_oracle(w, 1, 1, args.oracle_tokens, min_seconds=10.0, max_steps=30)
             line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
                                     "sample": desc}
         print(json.dumps(line), flush=True)
@@ -332,8 +387,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="b256", choices=sorted(si.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--oracle-tokens", type=int, default=12000,
-                    help="cached tokens in the oracle's bounded sample")
+    ap.add_argument("--oracle-tokens", type=int, default=40000,
+                    help="cached tokens in the cpu_baseline leg's bounded sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":

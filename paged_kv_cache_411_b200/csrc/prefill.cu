@@ -10,20 +10,21 @@
 //
 // One CTA computes one tile of 128 query rows x one head (FlashAttention
 // order, online softmax over 128-key tiles):
-//   * warp 4 (producer) loads the Q tile once and streams K and V tiles into a
+//   * warp 8 (producer) loads the Q tile once and streams K and V tiles into a
 //     two-stage ring with TMA: a K/V tile of 128 keys is gathered from the
 //     paged pool with one 3-D box per physical block ([box rows][1 head][64
 //     dims], 128-byte swizzle), landing directly in the canonical UMMA layout;
-//   * warp 5 (one elected thread) issues tcgen05.mma: S = Q K^T (A and B
+//   * warp 9 (one elected thread) issues tcgen05.mma: S = Q K^T (A and B
 //     K-major) into a double-buffered fp32 TMEM tile, and O_j = P_j V_j (B
 //     MN-major straight from the V tile) into a second double-buffered TMEM
 //     tile; completions are signalled with tcgen05.commit on mbarriers;
-//   * warps 0-3 (one thread per query row = one TMEM lane) read S with
-//     tcgen05.ld, apply the causal mask, run the online softmax in fp32
-//     (exp2 of prescaled logits), write P as fp16 into shared memory in the
-//     swizzled K-major layout the next MMA reads, and fold O_j into a
-//     register accumulator with the running rescale one tile behind, so the
-//     MMA of tile j+1 overlaps the softmax of tile j.
+//   * warps 0-7 (two threads per query row = per TMEM lane, each owning half
+//     of the columns) read S with tcgen05.ld, apply the causal mask on the
+//     diagonal tiles, agree on the row max through shared memory, run the
+//     online softmax in fp32 (exp2 of prescaled logits), write P as fp16 into
+//     shared memory in the swizzled K-major layout the next MMA reads, and
+//     fold O_j into a register accumulator with the running rescale one tile
+//     behind, so the MMA of tile j+1 overlaps the softmax of tile j.
 // Keys past the tile's last query position are masked; rows of V past the
 // sequence end are zeroed before P.V so stale or poisoned pool rows never
 // reach the MMA.  Every wait is bounded; on a timeout the CTA records
@@ -37,9 +38,10 @@ namespace pagedkv {
 namespace {
 
 constexpr int kTile = 128;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kThreadsP = 6 * 32;
+constexpr int kSoftmaxWarps = 8;          // two warpgroups: each owns half of the S / O columns
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreadsP = 10 * 32;
 constexpr float kLog2eP = 1.4426950408889634f;
 
 struct PrefillParams {
@@ -63,11 +65,12 @@ struct PCfg {
     static constexpr size_t kOffV = kOffK + size_t(kStages) * kOpBytes;
     static constexpr size_t kOffP = kOffV + size_t(kStages) * kOpBytes;
     static constexpr size_t kOffBar = kOffP + 2 * kChunkBytes;    // P: 128 rows x 128 keys fp16
-    static constexpr int kNumBars = 18;
+    static constexpr int kNumBars = 21;
     static constexpr size_t kOffSlot = kOffBar + kNumBars * 8;
+    static constexpr size_t kOffRed = kOffSlot + 64;                 // row-max exchange [2][2][128] + row sums [2][128]
     // Every CTA takes all 512 TMEM columns, so the request is kept above half the SM's shared
     // memory: one CTA per SM, and tcgen05.alloc never has to wait for a neighbour.
-    static constexpr size_t kSmemUsed = kOffSlot + 64 + 1024;
+    static constexpr size_t kSmemUsed = kOffRed + 6 * 128 * 4 + 1024;
     static constexpr size_t kSmemBytes = kSmemUsed > 120 * 1024 ? kSmemUsed : 120 * 1024;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColS = 0;                          // S buffers: columns 0 and 128
@@ -103,6 +106,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint64_t* o_full = bars + 13;    // [2]
     uint64_t* o_empty = bars + 15;   // [2]
     uint64_t* drain = bars + 17;
+    uint64_t* red_bar = bars + 18;   // [2] row-max exchange between the two softmax warpgroups
+    uint64_t* sum_bar = bars + 20;   // final row-sum exchange
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffSlot);
     volatile int* info = reinterpret_cast<volatile int*>(smem + C::kOffSlot + 16);   // b, qt, abort
 
@@ -140,13 +145,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&v_full[i], 1);
             mbar_init(&kv_empty[i], 1);
             mbar_init(&s_full[i], 1);
-            mbar_init(&s_empty[i], 4);
+            mbar_init(&s_empty[i], kSoftmaxWarps);
             mbar_init(&o_full[i], 1);
-            mbar_init(&o_empty[i], 4);
+            mbar_init(&o_empty[i], kSoftmaxWarps);
         }
-        mbar_init(p_full, 4);
+        mbar_init(p_full, kSoftmaxWarps);
         mbar_init(p_empty, 1);
         mbar_init(drain, 1);
+        mbar_init(&red_bar[0], kSoftmaxWarps);
+        mbar_init(&red_bar[1], kSoftmaxWarps);
+        mbar_init(sum_bar, kSoftmaxWarps);
         mbar_init_fence();
     }
     __syncthreads();
@@ -288,58 +296,70 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         __syncwarp();
     } else {
         // ======================================================= softmax warps
-        const int t = threadIdx.x;                    // query row within the tile = TMEM lane
-        const int row_in_req = qt * kTile + t;
+        // Thread (warpgroup g, row r): row r of the tile (TMEM lane r), columns g*64 .. g*64+63 of S
+        // and g*D/2 .. (g+1)*D/2-1 of O.  The two threads of a row agree on the running max through
+        // shared memory once per tile; each keeps a partial row sum, added at the end.
+        const int g = warp >> 2;
+        const int r = (warp & 3) * 32 + lane;
+        const int row_in_req = qt * kTile + r;
         const bool row_valid = row_in_req < L;
         const int row_pos = min(ctx + row_in_req, kv_len - 1);
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        const int tile_pos0 = ctx + qt * kTile;          // smallest query position in the tile
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        constexpr int DH = D / 2;
+        float* red = reinterpret_cast<float*>(smem + C::kOffRed);    // [parity][g][row], then sums [g][row]
         const float qs = p.qscale;
-        float acc[D];
+        float acc[DH];
 #pragma unroll
-        for (int i = 0; i < D; ++i) acc[i] = 0.f;
+        for (int i = 0; i < DH; ++i) acc[i] = 0.f;
         float m = -INFINITY, l = 0.f, alpha_prev = 0.f;
         bool ok = true;
         for (int j = 0; j < n_tiles && ok; ++j) {
             if (!(ok = mbar_wait(&s_full[j & 1], (j >> 1) & 1))) break;
             tc_fence_after_sync();
             const int key0 = j * kTile;
-            const uint32_t sa = lane_base + C::kColS + (j & 1) * kTile;
-            float mx = -INFINITY;
+            const bool diag = key0 + kTile - 1 > tile_pos0;          // some key of the tile is masked
+            const uint32_t sa = lane_base + C::kColS + (j & 1) * kTile + g * 64;
+            float sv[64];
+            {
+                float v0[32], v1[32];
+                tmem_ld_32cols(sa, v0);
+                tmem_ld_32cols(sa + 32, v1);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float v[32];
-                tmem_ld_32cols(sa + c * 32, v);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float s = key0 + c * 32 + i > row_pos ? -INFINITY : v[i] * qs;
-                    mx = fmaxf(mx, s);
-                }
+                for (int i = 0; i < 32; ++i) { sv[i] = v0[i]; sv[32 + i] = v1[i]; }
             }
+            if (diag) {
+#pragma unroll
+                for (int i = 0; i < 64; ++i)
+                    if (key0 + g * 64 + i > row_pos) sv[i] = -INFINITY;
+            }
+            float mx = sv[0];
+#pragma unroll
+            for (int i = 1; i < 64; ++i) mx = fmaxf(mx, sv[i]);
+            // raw scores: scale > 0 keeps the order, so the max is taken before scaling
+            float* rm = red + (j & 1) * 256;
+            rm[g * 128 + r] = mx;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&red_bar[j & 1]);
+            if (!(ok = mbar_wait(&red_bar[j & 1], (j >> 1) & 1))) break;
+            mx = fmaxf(mx, rm[(g ^ 1) * 128 + r]) * qs;
             const float m_new = fmaxf(m, mx);
             const float m_use = m_new == -INFINITY ? 0.f : m_new;
             const float alpha = exp2f(m - m_use);
             if (!(ok = mbar_wait(p_empty, (j & 1) ^ 1))) break;
             float rs = 0.f;
+            uint8_t* prow = sP + g * C::kChunkBytes + r * 128;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {                 // 16 keys = two 16-byte units of P per step
-                float v[16];
-                tmem_ld_16cols(sa + c * 16, v);
-                uint32_t pk[8];
+            for (int u = 0; u < 8; ++u) {                     // 8 keys = one 16-byte unit of P
+                uint32_t pk[4];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int k = key0 + c * 16 + 2 * i;
-                    const float p0 = k > row_pos ? 0.f : exp2f(v[2 * i] * qs - m_use);
-                    const float p1 = k + 1 > row_pos ? 0.f : exp2f(v[2 * i + 1] * qs - m_use);
+                for (int i = 0; i < 4; ++i) {
+                    const float p0 = exp2f(fmaf(sv[8 * u + 2 * i], qs, -m_use));
+                    const float p1 = exp2f(fmaf(sv[8 * u + 2 * i + 1], qs, -m_use));
                     rs += p0 + p1;
                     pk[i] = f2_to_h2(p0, p1);
                 }
-                uint8_t* prow = sP + (c >> 2) * C::kChunkBytes + t * 128;
-#pragma unroll
-                for (int uu = 0; uu < 2; ++uu) {
-                    const int u = (c & 3) * 2 + uu;
-                    st_shared_u4(prow + ((u ^ (t & 7)) * 16),
-                                 make_uint4(pk[4 * uu], pk[4 * uu + 1], pk[4 * uu + 2], pk[4 * uu + 3]));
-                }
+                st_shared_u4(prow + ((u ^ (r & 7)) * 16), make_uint4(pk[0], pk[1], pk[2], pk[3]));
             }
             tc_fence_before_sync();
             __syncwarp();
@@ -347,12 +367,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (j == n_tiles - 1 && kv_len < key0 + kTile) {
                 // rows of V past the sequence end may hold anything: zero them before P.V reads them
                 if (!(ok = mbar_wait(&v_full[j & 1], (j >> 1) & 1))) break;
-                if (key0 + t >= kv_len) {
-                    uint8_t* vrow = sV + (j & 1) * C::kOpBytes + t * 128;
+                if (key0 + r >= kv_len) {
+                    uint8_t* vrow = sV + (j & 1) * C::kOpBytes + r * 128;
 #pragma unroll
                     for (int c = 0; c < C::kChunks; ++c)
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) st_shared_u4(vrow + c * C::kChunkBytes + u * 16, make_uint4(0, 0, 0, 0));
+                        for (int u = 0; u < 8 / 2; ++u)
+                            st_shared_u4(vrow + c * C::kChunkBytes + (g * 4 + u) * 16, make_uint4(0, 0, 0, 0));
                 }
             }
             fence_proxy_async_smem();
@@ -363,9 +384,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const int jp = j - 1;
                 if (!(ok = mbar_wait(&o_full[jp & 1], (jp >> 1) & 1))) break;
                 tc_fence_after_sync();
-                const uint32_t oa = lane_base + C::kColO + (jp & 1) * D;
+                const uint32_t oa = lane_base + C::kColO + (jp & 1) * D + g * DH;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = 0; c < DH / 32; ++c) {
                     float v[32];
                     tmem_ld_32cols(oa + c * 32, v);
 #pragma unroll
@@ -384,27 +405,34 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             ok = mbar_wait(&o_full[jp & 1], (jp >> 1) & 1);
             if (ok) {
                 tc_fence_after_sync();
-                const uint32_t oa = lane_base + C::kColO + (jp & 1) * D;
+                const uint32_t oa = lane_base + C::kColO + (jp & 1) * D + g * DH;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = 0; c < DH / 32; ++c) {
                     float v[32];
                     tmem_ld_32cols(oa + c * 32, v);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) acc[c * 32 + i] = fmaf(acc[c * 32 + i], alpha_prev, v[i]);
                 }
-                if (row_valid) {
-                    const float inv = 1.f / l;
-                    __half* orow = p.out + (static_cast<int64_t>(q0 + t) * p.H + h) * D;
+            }
+        }
+        // both threads of a row add their partial sums (every softmax thread reaches this barrier)
+        float* rsum = red + 512;
+        rsum[g * 128 + r] = l;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sum_bar);
+        if (ok) ok = mbar_wait(sum_bar, 0);
+        l += rsum[(g ^ 1) * 128 + r];
+        if (ok && row_valid) {
+            const float inv = 1.f / l;
+            __half* orow = p.out + (static_cast<int64_t>(q0 + r) * p.H + h) * D + g * DH;
 #pragma unroll
-                    for (int c = 0; c < D / 8; ++c) {
-                        uint4 o;
-                        o.x = f2_to_h2(acc[8 * c + 0] * inv, acc[8 * c + 1] * inv);
-                        o.y = f2_to_h2(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv);
-                        o.z = f2_to_h2(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv);
-                        o.w = f2_to_h2(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv);
-                        *reinterpret_cast<uint4*>(orow + 8 * c) = o;
-                    }
-                }
+            for (int c = 0; c < DH / 8; ++c) {
+                uint4 o;
+                o.x = f2_to_h2(acc[8 * c + 0] * inv, acc[8 * c + 1] * inv);
+                o.y = f2_to_h2(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv);
+                o.z = f2_to_h2(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv);
+                o.w = f2_to_h2(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv);
+                *reinterpret_cast<uint4*>(orow + 8 * c) = o;
             }
         }
         if (!ok) abort_now();
