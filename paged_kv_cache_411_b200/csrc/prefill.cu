@@ -65,7 +65,7 @@ struct PCfg {
     static constexpr size_t kOffV = kOffK + size_t(kStages) * kOpBytes;
     static constexpr size_t kOffP = kOffV + size_t(kStages) * kOpBytes;
     static constexpr size_t kOffBar = kOffP + 2 * kChunkBytes;    // P: 128 rows x 128 keys fp16
-    static constexpr int kNumBars = 21;
+    static constexpr int kNumBars = 23;
     static constexpr size_t kOffSlot = kOffBar + kNumBars * 8;
     static constexpr size_t kOffRed = kOffSlot + 64;                 // row-max exchange [2][2][128] + row sums [2][128]
     // Every CTA takes all 512 TMEM columns, so the request is kept above half the SM's shared
@@ -98,7 +98,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint64_t* q_full = bars + 0;
     uint64_t* k_full = bars + 1;     // [2]
     uint64_t* v_full = bars + 3;     // [2]
-    uint64_t* kv_empty = bars + 5;   // [2]
+    uint64_t* k_empty = bars + 5;    // [2] released by the S MMA
+    uint64_t* v_empty = bars + 21;   // [2] released by the P.V MMA
     uint64_t* s_full = bars + 7;     // [2]
     uint64_t* s_empty = bars + 9;    // [2]
     uint64_t* p_full = bars + 11;
@@ -143,7 +144,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int i = 0; i < 2; ++i) {
             mbar_init(&k_full[i], 1);
             mbar_init(&v_full[i], 1);
-            mbar_init(&kv_empty[i], 1);
+            mbar_init(&k_empty[i], 1);
+            mbar_init(&v_empty[i], 1);
             mbar_init(&s_full[i], 1);
             mbar_init(&s_empty[i], kSoftmaxWarps);
             mbar_init(&o_full[i], 1);
@@ -197,11 +199,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         const int br = p.box_rows;
         const int64_t tbase = static_cast<int64_t>(b) * p.max_blocks;
-        int issued_last = -1;
+        int k_last = -1, v_last = -1;     // last tiles whose K / V copies were issued
         for (int j = 0; j < n_tiles; ++j) {
             const int st = j & 1;
-            if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1)) { abort_now(); break; }
-            if (info[2]) break;
             const int key0 = j * kTile;
             const int nkeys = min(kTile, kv_len - key0);
             const int nbox = (nkeys + br - 1) / br;
@@ -215,11 +215,25 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
             }
             const uint32_t bytes = static_cast<uint32_t>(nbox * br * 128 * C::kChunks);
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&k_full[st], bytes);
-                mbar_arrive_expect_tx(&v_full[st], bytes);
-            }
+            // K tile: its stage frees as soon as S of the tile two back has been computed
+            if (!mbar_wait(&k_empty[st], ((j >> 1) & 1) ^ 1)) { abort_now(); break; }
+            if (info[2]) break;
+            if (lane == 0) mbar_arrive_expect_tx(&k_full[st], bytes);
             uint8_t* dk = sK + st * C::kOpBytes;
+            for (int i = 0; i < nbox; ++i) {
+                const int bi = __shfl_sync(0xffffffffu, bid, i);
+                if (lane == 0) {
+                    const int key = key0 + i * br;
+                    const int row = bi * p.bs + key % p.bs;
+#pragma unroll
+                    for (int c = 0; c < C::kChunks; ++c)
+                        tma_load_3d(dk + c * C::kChunkBytes + i * br * 128, &tm_k, &k_full[st], c * 64, h, row, pol);
+                }
+            }
+            // V tile: its stage frees when P.V of the tile two back has completed
+            k_last = j;
+            if (!mbar_wait(&v_empty[st], ((j >> 1) & 1) ^ 1)) { abort_now(); break; }
+            if (lane == 0) mbar_arrive_expect_tx(&v_full[st], bytes);
             uint8_t* dv = sV + st * C::kOpBytes;
             for (int i = 0; i < nbox; ++i) {
                 const int bi = __shfl_sync(0xffffffffu, bid, i);
@@ -227,20 +241,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     const int key = key0 + i * br;
                     const int row = bi * p.bs + key % p.bs;
 #pragma unroll
-                    for (int c = 0; c < C::kChunks; ++c) {
-                        tma_load_3d(dk + c * C::kChunkBytes + i * br * 128, &tm_k, &k_full[st], c * 64, h, row, pol);
+                    for (int c = 0; c < C::kChunks; ++c)
                         tma_load_3d(dv + c * C::kChunkBytes + i * br * 128, &tm_v, &v_full[st], c * 64, h, row, pol);
-                    }
                 }
             }
-            issued_last = j;
+            v_last = j;
         }
-        if (info[2] && issued_last >= 0) {
+        if (info[2]) {
             // unwind: let the copies this warp issued into each stage land
-            for (int j = max(0, issued_last - 1); j <= issued_last; ++j) {
-                (void)mbar_wait(&k_full[j & 1], (j >> 1) & 1);
-                (void)mbar_wait(&v_full[j & 1], (j >> 1) & 1);
-            }
+            for (int j = max(0, k_last - 1); j <= k_last; ++j) (void)mbar_wait(&k_full[j & 1], (j >> 1) & 1);
+            for (int j = max(0, v_last - 1); j <= v_last; ++j) (void)mbar_wait(&v_full[j & 1], (j >> 1) & 1);
         }
     } else if (warp == kMmaWarp) {
         // ======================================================= MMA issuer
@@ -263,6 +273,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                 kk > 0);
                 }
                 umma_commit(&s_full[j & 1]);
+                umma_commit(&k_empty[st]);
                 return true;
             };
             if (ok) ok = issue_s(0);
@@ -284,7 +295,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
                 umma_commit(&o_full[j & 1]);
                 umma_commit(p_empty);
-                umma_commit(&kv_empty[st]);
+                umma_commit(&v_empty[st]);
             }
             if (!ok) {
                 abort_now();
