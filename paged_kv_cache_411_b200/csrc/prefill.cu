@@ -10,10 +10,12 @@
 //
 // One CTA computes one tile of 128 query rows x one head (FlashAttention
 // order, online softmax over 128-key tiles):
-//   * warp 8 (producer) loads the Q tile once and streams K and V tiles into a
-//     two-stage ring with TMA: a K/V tile of 128 keys is gathered from the
-//     paged pool with one 3-D box per physical block ([box rows][1 head][64
-//     dims], 128-byte swizzle), landing directly in the canonical UMMA layout;
+//   * warp 8 (producer) loads the Q tile once and streams K and V tiles into
+//     two-stage rings with TMA: a K/V tile of 128 keys is gathered from the
+//     paged pool with one 3-D box per physical block and 64-dim chunk ([box
+//     rows][1 head][64 dims], 128-byte swizzle), landing directly in the
+//     canonical UMMA layout; each lane issues its own block's boxes, and the
+//     next tile's block ids are read while the current tile's copies go out;
 //   * warp 9 (one elected thread) issues tcgen05.mma: S = Q K^T (A and B
 //     K-major) into a double-buffered fp32 TMEM tile, and O_j = P_j V_j (B
 //     MN-major straight from the V tile) into a second double-buffered TMEM
@@ -200,52 +202,55 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int br = p.box_rows;
         const int64_t tbase = static_cast<int64_t>(b) * p.max_blocks;
         int k_last = -1, v_last = -1;     // last tiles whose K / V copies were issued
-        for (int j = 0; j < n_tiles; ++j) {
-            const int st = j & 1;
+        // Block ids of a tile: lane i holds the physical block of the tile's i-th box.  The ids of
+        // tile j+1 are loaded while tile j's copies are issued, so the table read never stalls a tile.
+        auto load_ids = [&](int j) -> int {
             const int key0 = j * kTile;
-            const int nkeys = min(kTile, kv_len - key0);
-            const int nbox = (nkeys + br - 1) / br;
+            const int nbox = (min(kTile, kv_len - key0) + br - 1) / br;
             int bid = 0;
-            if (lane < nbox) {
-                const int key = key0 + lane * br;
-                bid = p.block_tables[tbase + key / p.bs];
+            if (j < n_tiles && lane < nbox) {
+                bid = p.block_tables[tbase + (key0 + lane * br) / p.bs];
                 if (bid < 0 || bid >= p.num_blocks) {
                     flag_error(p.err_flag, PA_DEVCHK_BLOCK_ID);
                     bid = 0;
                 }
             }
+            return bid;
+        };
+        int bid = load_ids(0);
+        for (int j = 0; j < n_tiles; ++j) {
+            const int st = j & 1;
+            const int key0 = j * kTile;
+            const int nkeys = min(kTile, kv_len - key0);
+            const int nbox = (nkeys + br - 1) / br;
+            const int bid_next = load_ids(j + 1);
             const uint32_t bytes = static_cast<uint32_t>(nbox * br * 128 * C::kChunks);
+            // Each lane issues its own boxes: the copies of a tile go out in parallel.
+            const int row = bid * p.bs + (key0 + lane * br) % p.bs;
             // K tile: its stage frees as soon as S of the tile two back has been computed
             if (!mbar_wait(&k_empty[st], ((j >> 1) & 1) ^ 1)) { abort_now(); break; }
             if (info[2]) break;
             if (lane == 0) mbar_arrive_expect_tx(&k_full[st], bytes);
-            uint8_t* dk = sK + st * C::kOpBytes;
-            for (int i = 0; i < nbox; ++i) {
-                const int bi = __shfl_sync(0xffffffffu, bid, i);
-                if (lane == 0) {
-                    const int key = key0 + i * br;
-                    const int row = bi * p.bs + key % p.bs;
+            __syncwarp();
+            if (lane < nbox) {
+                uint8_t* dk = sK + st * C::kOpBytes + lane * br * 128;
 #pragma unroll
-                    for (int c = 0; c < C::kChunks; ++c)
-                        tma_load_3d(dk + c * C::kChunkBytes + i * br * 128, &tm_k, &k_full[st], c * 64, h, row, pol);
-                }
+                for (int c = 0; c < C::kChunks; ++c)
+                    tma_load_3d(dk + c * C::kChunkBytes, &tm_k, &k_full[st], c * 64, h, row, pol);
             }
-            // V tile: its stage frees when P.V of the tile two back has completed
             k_last = j;
+            // V tile: its stage frees when P.V of the tile two back has completed
             if (!mbar_wait(&v_empty[st], ((j >> 1) & 1) ^ 1)) { abort_now(); break; }
             if (lane == 0) mbar_arrive_expect_tx(&v_full[st], bytes);
-            uint8_t* dv = sV + st * C::kOpBytes;
-            for (int i = 0; i < nbox; ++i) {
-                const int bi = __shfl_sync(0xffffffffu, bid, i);
-                if (lane == 0) {
-                    const int key = key0 + i * br;
-                    const int row = bi * p.bs + key % p.bs;
+            __syncwarp();
+            if (lane < nbox) {
+                uint8_t* dv = sV + st * C::kOpBytes + lane * br * 128;
 #pragma unroll
-                    for (int c = 0; c < C::kChunks; ++c)
-                        tma_load_3d(dv + c * C::kChunkBytes + i * br * 128, &tm_v, &v_full[st], c * 64, h, row, pol);
-                }
+                for (int c = 0; c < C::kChunks; ++c)
+                    tma_load_3d(dv + c * C::kChunkBytes, &tm_v, &v_full[st], c * 64, h, row, pol);
             }
             v_last = j;
+            bid = bid_next;
         }
         if (info[2]) {
             // unwind: let the copies this warp issued into each stage land
