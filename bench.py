@@ -124,6 +124,16 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def pool_stats(ds):
+    """Measured internal fragmentation of the pool vs the page's (block_size / 2) / avg_len estimate."""
+    st = ds.alloc.stats()
+    w = ds.workload
+    ctx = int(ds.seq_lens_host.astype(np.int64).sum())
+    return {"block_size": w.block_size, "num_blocks": st["num_blocks"], "used_blocks": st["num_used"],
+            "waste_tokens": st["waste_tokens"], "waste_frac": round(st["waste_tokens"] / max(1, ctx), 5),
+            "page_estimate_frac": round((w.block_size / 2) / (ctx / w.num_seqs), 5)}
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -222,6 +232,8 @@ def run_reference(args):
     if rank != 0:
         return 0
     w = si.get(args.workload)
+    if args.block_size:
+        w = si.with_block_size(w, args.block_size)
     per_step = oracle_tokens_for(w, args.steps + args.warmup, 120.0)
     gbs, dt, desc, threads = time_oracle(w, args.steps, args.warmup, per_step)
     line = {
@@ -253,6 +265,8 @@ def run_ours(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
     w = si.get(args.workload)
+    if args.block_size:
+        w = si.with_block_size(w, args.block_size)
     ds = pwl.build(w, device=device)
     S, H, D = ds.q.shape
     T = ds.k_step.shape[0]
@@ -359,6 +373,7 @@ def run_ours(args):
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(1e3 * e2e_max / args.steps, 4)},
             "gpu_launches": args.steps * (4 + (1 if pout is not None else 0)),
+            "kv_pool": pool_stats(ds),
             "clocks": clk.summary(),
         }
         if pout is not None:
@@ -387,6 +402,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="b256", choices=sorted(si.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--block-size", type=int, default=0,
+                    help="run the workload's requests with this block size instead (block-size sweep)")
     ap.add_argument("--oracle-tokens", type=int, default=40000,
                     help="cached tokens in the cpu_baseline leg's bounded sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -224,6 +224,13 @@ def get(name: str) -> Workload:
     return WORKLOADS[name]()
 
 
+def with_block_size(w: Workload, block_size: int) -> Workload:
+    """The same requests and draws with another block size (for block-size sweeps)."""
+    if block_size == w.block_size:
+        return w
+    return dataclasses.replace(w, block_size=int(block_size), name=f"{w.name}__bs{block_size}")
+
+
 def garbage_block_ids(seed: int, shape, num_blocks: int) -> np.ndarray:
     """In-range but wrong block ids used to fill the padding of packed block tables in tests."""
     return rng(seed, "garbage").integers(0, num_blocks, size=shape).astype(np.int32)

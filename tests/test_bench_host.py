@@ -1,0 +1,99 @@
+"""Host-side logic of bench.py (no GPU): algorithmic byte and FLOP counts, the oracle
+sample bound, reference-arm rank gating, and the multi-rank reduction (max of times,
+sum of bytes) run as two gloo ranks on the CPU."""
+import io
+import json
+import os
+import socket
+import sys
+from contextlib import redirect_stdout
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+import synth_inputs as si
+
+
+def test_step_bytes_tiny():
+    w = si.tiny()
+    dec, rs, pre = bench.step_bytes(w, w.decode_lens, 3, 4)
+    H, D = 4, 64
+    kv = sum(w.decode_lens) * H * D * 2 * 2
+    assert dec == kv + 2 * 4 * H * D * 2 + (1 + 1 + 2 + 3) * 4 + 4 * 4
+    assert rs == 4 * H * D * 2 * 2 * 2 + 4 * 8
+    assert pre == 0
+
+
+def test_prefill_flops_mixed():
+    # 512 rows after 1536 cached tokens: 917,760 visible pairs per head, 4 * 32 * 128 flops each
+    w = si.get("mixed")
+    assert bench.prefill_flops(w) == 917_760 * 4 * 32 * 128 == 15_036_579_840
+
+
+def test_oracle_sample_is_bounded_and_seeded():
+    w = si.get("b256")
+    a = bench.oracle_sample_seqs(w, 12000)
+    b = bench.oracle_sample_seqs(w, 12000)
+    assert a == b and a == sorted(a)
+    tot = sum(w.decode_lens[s] for s in a)
+    assert tot <= 12000 + max(w.decode_lens)
+
+
+def test_reference_arm_runs_on_rank0_only(monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    f = io.StringIO()
+    with redirect_stdout(f):
+        rc = bench.main(["--impl", "reference", "--steps", "1", "--warmup", "0", "--workload", "tiny"])
+    assert rc == 0 and f.getvalue() == ""
+
+
+def test_reference_arm_line_on_rank0(monkeypatch):
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    f = io.StringIO()
+    with redirect_stdout(f):
+        rc = bench.main(["--impl", "reference", "--steps", "2", "--warmup", "1", "--workload", "tiny"])
+    line = json.loads(f.getvalue().strip().splitlines()[-1])
+    assert rc == 0 and line["impl"] == "reference" and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["unit"] == "GB/s" and line["higher_is_better"] is True
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        mx, sm = bench.reduce_max_sum(10.0 + 5 * rank, 100.0 * (rank + 1), torch.device("cpu"))
+        q.put((rank, mx, sm))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_reduce_max_sum_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=5) for _ in range(2))
+    # every rank sees the max of the times and the sum of the bytes
+    assert res == [(0, 15.0, 300.0), (1, 15.0, 300.0)]
+
+
+def test_reduce_is_identity_without_process_group():
+    assert bench.reduce_max_sum(3.0, 7.0, torch.device("cpu")) == (3.0, 7.0)

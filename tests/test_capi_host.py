@@ -175,3 +175,19 @@ def test_workload_replay_matches_oracle(name):
             ot = o.block_tables[index]
             pos = np.arange(pos0, pos0 + len(sl))
             assert np.array_equal(sl, ot[pos // w.block_size].astype(np.int64) * w.block_size + pos % w.block_size)
+
+
+@pytest.mark.parametrize("bs", [8, 16, 32, 64])
+def test_internal_waste_matches_page_estimate(bs):
+    """Block-size trade-off (page §3.4): each request wastes < block_size slots of its last block;
+    on the ragged batch-256 lengths the mean waste per request is close to (bs - 1) / 2, the page's
+    bs / 2 estimate, measured from the C++ allocator's counters."""
+    w = si.with_block_size(si.get("b256"), bs)
+    r = pwl.replay(w)
+    st = r.alloc.stats()
+    S = w.num_seqs
+    per_req = st["waste_tokens"] / S
+    assert abs(per_req - (bs - 1) / 2) < 0.15 * bs
+    _, t, lens = r.alloc.pack(np.arange(S), max(-(-n // bs) for n in w.decode_lens))
+    waste = (t >= 0).sum(axis=1) * bs - lens
+    assert (waste >= 0).all() and (waste < bs).all() and waste.sum() == st["waste_tokens"]
