@@ -137,7 +137,9 @@ pa_status pa_alloc_append_tokens(pa_alloc* a, int64_t req, int32_t n, int64_t* s
 pa_status pa_alloc_fork(pa_alloc* a, int64_t src, int64_t dst, int32_t prefix_tokens);
 
 /* [CB-PA] §3.2 free: decrement the refcount of every block of req's table in
- * order; push the ones reaching zero.  Freeing an unknown id is a no-op (PA_OK). */
+ * order; push the ones reaching zero on the free list in table order (blocks
+ * registered by the prefix cache are parked in its LRU instead, see below).
+ * Freeing an unknown id is a no-op (PA_OK). */
 pa_status pa_alloc_free(pa_alloc* a, int64_t req);
 
 /* Copy req's block table into out[0..cap).  *len_out (nullable) = its length.
@@ -167,6 +169,38 @@ pa_status pa_alloc_refcount(const pa_alloc* a, int32_t block, int32_t* out);
 /* Copy the free list (bottom to top; the next pop takes the last entry).
  * Errors: INVALID_ARG (cap < length; *len_out still set). */
 pa_status pa_alloc_free_list(const pa_alloc* a, int32_t* out, int32_t cap, int32_t* len_out);
+
+/* ---- automatic prefix caching ([CB-PA] §4.1 content-hashed shared blocks,
+ * §4.2 Automatic Prefix Caching with an LRU of recently used blocks) ----------
+ *
+ * A full block's content is identified exactly by its whole token prefix (a
+ * prefix-trie node: parent prefix + the block's block_size token ids).  A
+ * registered block whose refcount drops to zero is parked in an LRU instead
+ * of the free list; any take (allocate, append, allocate_cached) pops the free
+ * list first and evicts the least recently parked block when it is empty.
+ * Requests are parked last block first, so a prefix outlives its extensions. */
+
+typedef struct {
+    int64_t cached_blocks;     /* blocks registered under a prefix node           */
+    int64_t evictable_blocks;  /* registered blocks with refcount 0 (the LRU)      */
+    int64_t hit_blocks;        /* blocks reused by allocate_cached so far          */
+    int64_t evictions;         /* parked blocks taken back for new content         */
+    int64_t prefix_nodes;      /* distinct block prefixes seen                     */
+} pa_cache_stats_t;
+
+/* Allocate `req` for tokens[0..num_tokens) (host int32 token ids), reusing the
+ * cached blocks of the longest cached prefix of whole blocks (refcount + 1,
+ * taken out of the LRU) and taking new blocks for the rest; the new full
+ * blocks are registered.  *cached_tokens_out (nullable) = reused blocks *
+ * block_size: the KV the caller need not recompute or write.  All-or-nothing.
+ * Errors: EXISTS, OOM (nothing changes), INVALID_ARG. */
+pa_status pa_alloc_allocate_cached(pa_alloc* a, int64_t req, const int32_t* tokens, int32_t num_tokens,
+                                   int32_t* cached_tokens_out);
+/* Prefix-cache counters. */
+pa_status pa_alloc_cache_stats(const pa_alloc* a, pa_cache_stats_t* out);
+/* Copy the LRU of parked blocks, least recently parked first (the next
+ * eviction takes out[0]).  Errors: INVALID_ARG (cap < length; *len_out set). */
+pa_status pa_alloc_evictable_list(const pa_alloc* a, int32_t* out, int32_t cap, int32_t* len_out);
 
 /* ---- device kernels -------------------------------------------------------- */
 

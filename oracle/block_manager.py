@@ -60,14 +60,10 @@ class BlockManager:
         if req in self.block_tables:
             return EXISTS
         n = blocks_needed(num_tokens, self.block_size)
-        if len(self.free_blocks) < n:
+        if self._available() < n:
             self.oom_count += 1
             return OOM
-        blocks = []
-        for _ in range(n):
-            b = self.free_blocks.pop()
-            self.refcount[b] += 1
-            blocks.append(b)
+        blocks = [self._take() for _ in range(n)]
         self.block_tables[req] = blocks
         self.seq_lens[req] = num_tokens
         return OK
@@ -80,12 +76,10 @@ class BlockManager:
         table = self.block_tables[req]
         cur = self.seq_lens[req]
         if cur % self.block_size == 0:
-            if not self.free_blocks:
+            if self._available() == 0:
                 self.oom_count += 1
                 return OOM, None
-            b = self.free_blocks.pop()
-            self.refcount[b] += 1
-            table.append(b)
+            table.append(self._take())
         self.seq_lens[req] = cur + 1
         return OK, self.slot(req, cur)
 
@@ -97,7 +91,7 @@ class BlockManager:
             return NOT_FOUND, []
         cur = self.seq_lens[req]
         extra = blocks_needed(cur + n, self.block_size) - len(self.block_tables[req])
-        if extra > len(self.free_blocks):
+        if extra > self._available():
             self.oom_count += 1
             return OOM, []
         slots = []
@@ -127,13 +121,25 @@ class BlockManager:
     def free(self, req: int) -> str:
         if req not in self.block_tables:
             return OK
-        for b in self.block_tables[req]:
-            self.refcount[b] -= 1
-            if self.refcount[b] == 0:
-                self.free_blocks.append(b)
+        self._release(self.block_tables[req])
         del self.block_tables[req]
         del self.seq_lens[req]
         return OK
+
+    # ---- free-list primitives (the prefix cache overrides them) -------------
+    def _available(self) -> int:
+        return len(self.free_blocks)
+
+    def _take(self) -> int:
+        b = self.free_blocks.pop()
+        self.refcount[b] += 1
+        return b
+
+    def _release(self, table) -> None:
+        for b in table:
+            self.refcount[b] -= 1
+            if self.refcount[b] == 0:
+                self.free_blocks.append(b)
 
     # ---- queries ----------------------------------------------------------
     def get_block_table(self, req: int):

@@ -19,7 +19,7 @@ import numpy as np
 from ._lib import (PA_DEVCHK_BLOCK_ID, PA_DEVCHK_QUERY_RANGE, PA_DEVCHK_SEQ_LEN, PA_DEVCHK_SLOT,
                    PA_DEVCHK_TIMEOUT, PA_ERR_CUDA, PA_ERR_DEVICE_CHECK, PA_ERR_EXISTS, PA_ERR_INVALID_ARG,
                    PA_ERR_NOT_FOUND, PA_ERR_OOM, PA_ERR_UNSUPPORTED, PA_OK, STATUS_NAMES, AllocStats,
-                   PagedKVError, check, last_error, lib)
+                   CacheStats, PagedKVError, check, last_error, lib)
 
 __all__ = [
     "BlockAllocator", "reshape_and_cache", "paged_attention_decode", "paged_attention_prefill_chunk",
@@ -123,6 +123,26 @@ class BlockAllocator:
         lib().pa_alloc_free_list(self._h, None, 0, byref(n))
         out = np.empty(n.value, dtype=np.int32)
         check(lib().pa_alloc_free_list(self._h, _i32p(out), n.value, byref(n)))
+        return out
+
+    # ---- automatic prefix caching
+    def allocate_cached(self, req: int, tokens):
+        """Returns (status, cached_tokens): blocks of the longest cached prefix are reused."""
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        n = c_int32(0)
+        st = lib().pa_alloc_allocate_cached(self._h, req, _i32p(t), len(t), byref(n))
+        return st, (n.value if st == PA_OK else 0)
+
+    def cache_stats(self) -> dict:
+        s = CacheStats()
+        check(lib().pa_alloc_cache_stats(self._h, byref(s)))
+        return s.as_dict()
+
+    def evictable_list(self) -> np.ndarray:
+        n = c_int32(0)
+        lib().pa_alloc_evictable_list(self._h, None, 0, byref(n))
+        out = np.empty(n.value, dtype=np.int32)
+        check(lib().pa_alloc_evictable_list(self._h, _i32p(out), n.value, byref(n)))
         return out
 
 

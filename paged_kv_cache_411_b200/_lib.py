@@ -52,6 +52,14 @@ class AllocStats(ctypes.Structure):
         return {k: getattr(self, k) for k, _ in self._fields_}
 
 
+class CacheStats(ctypes.Structure):
+    _fields_ = [("cached_blocks", c_int64), ("evictable_blocks", c_int64), ("hit_blocks", c_int64),
+                ("evictions", c_int64), ("prefix_nodes", c_int64)]
+
+    def as_dict(self):
+        return {k: getattr(self, k) for k, _ in self._fields_}
+
+
 _P = c_void_p
 _I32P = POINTER(c_int32)
 _I64P = POINTER(c_int64)
@@ -76,6 +84,9 @@ SIGNATURES = {
     "pa_alloc_stats": (c_int32, [_P, POINTER(AllocStats)]),
     "pa_alloc_refcount": (c_int32, [_P, c_int32, _I32P]),
     "pa_alloc_free_list": (c_int32, [_P, _I32P, c_int32, _I32P]),
+    "pa_alloc_allocate_cached": (c_int32, [_P, c_int64, _I32P, c_int32, _I32P]),
+    "pa_alloc_cache_stats": (c_int32, [_P, POINTER(CacheStats)]),
+    "pa_alloc_evictable_list": (c_int32, [_P, _I32P, c_int32, _I32P]),
     "pa_reshape_and_cache": (c_int32, [_P, _P, _P, _P, _P, c_int32, c_int32, c_int32, c_int32, c_int32, _P, _P]),
     "pa_decode_workspace_bytes": (c_size_t, [c_int32, c_int32, c_int32, c_int32, c_int32]),
     "pa_paged_attention_decode": (c_int32, [_P, _P, _P, _P, _P, _P, c_int32, c_int32, c_int32, c_int32, c_int32,

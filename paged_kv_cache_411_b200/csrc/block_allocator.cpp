@@ -13,9 +13,25 @@
 //   * a token's slot is table[pos / block_size] * block_size + pos % block_size
 //     (the address form of the page's §3.3 kernel).
 // Everything is O(1) per token except free, which is O(table length).
+//
+// Automatic prefix caching (§4.1 hashes the token content of blocks and keeps
+// identical blocks once; §4.2 keeps recently used blocks in an LRU):
+//   * a full block's content is identified exactly by a node of a prefix trie,
+//     node = intern(parent node, the block's block_size token ids), so two
+//     blocks match only when the whole token prefix up to their end matches;
+//   * allocate_cached reuses the cached blocks of the longest cached prefix
+//     (walking from the first block, stopping at the first miss), takes new
+//     blocks for the rest and registers the new full blocks; the partial last
+//     block stays private;
+//   * a registered block whose refcount drops to zero is not freed but parked
+//     in an LRU of evictable blocks (a request's blocks are parked last block
+//     first, so a prefix is always at least as recent as its extensions);
+//   * a take pops the free list, or, when it is empty, evicts the least
+//     recently used parked block (its cache entry is dropped).
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
+#include <list>
 #include <new>
 #include <unordered_map>
 #include <vector>
@@ -44,6 +60,27 @@ const char* last_error() { return g_last_error.c_str(); }
 
 using pagedkv::fail;
 
+namespace {
+
+struct PrefixKey {
+    int64_t parent;
+    std::vector<int32_t> tokens;
+    bool operator==(const PrefixKey& o) const { return parent == o.parent && tokens == o.tokens; }
+};
+
+struct PrefixKeyHash {
+    size_t operator()(const PrefixKey& k) const {
+        uint64_t h = 1469598103934665603ull ^ static_cast<uint64_t>(k.parent);
+        for (int32_t t : k.tokens) {
+            h ^= static_cast<uint32_t>(t);
+            h *= 1099511628211ull;
+        }
+        return static_cast<size_t>(h ^ (h >> 29));
+    }
+};
+
+}  // namespace
+
 struct pa_alloc {
     struct Request {
         std::vector<int32_t> table;
@@ -55,13 +92,65 @@ struct pa_alloc {
     std::vector<int32_t> refcount;
     std::unordered_map<int64_t, Request> reqs;
     int64_t oom_count = 0;
+    // prefix cache
+    std::unordered_map<PrefixKey, int64_t, PrefixKeyHash> trie;   // (parent node, tokens) -> node
+    std::unordered_map<int64_t, int32_t> cache;                    // node -> block
+    std::vector<int64_t> block_node;                               // block -> node, -1 if not registered
+    std::list<int32_t> lru;                                        // parked blocks, least recent first
+    std::vector<std::list<int32_t>::iterator> lru_pos;
+    std::vector<char> in_lru;
+    int64_t hit_blocks = 0, evictions = 0;
 
     int64_t blocks_for(int64_t tokens) const { return (tokens + block_size - 1) / block_size; }
+    int64_t available() const { return static_cast<int64_t>(free_list.size() + lru.size()); }
+    void unpark(int32_t b) {
+        lru.erase(lru_pos[b]);
+        in_lru[b] = 0;
+    }
     int32_t take() {
-        int32_t b = free_list.back();
-        free_list.pop_back();
+        int32_t b;
+        if (!free_list.empty()) {
+            b = free_list.back();
+            free_list.pop_back();
+        } else {
+            b = lru.front();
+            unpark(b);
+            cache.erase(block_node[b]);
+            block_node[b] = -1;
+            evictions += 1;
+        }
         refcount[b] += 1;
         return b;
+    }
+    // Drop one reference to every block of `table`; blocks reaching zero go to the free list
+    // (unregistered, table order) or are parked in the LRU (registered, last block first).
+    void release(const std::vector<int32_t>& table) {
+        std::vector<int32_t> zero;
+        for (int32_t b : table)
+            if (--refcount[b] == 0) zero.push_back(b);
+        for (int32_t b : zero)
+            if (block_node[b] < 0) free_list.push_back(b);
+        for (auto it = zero.rbegin(); it != zero.rend(); ++it) {
+            const int32_t b = *it;
+            if (block_node[b] >= 0) {
+                lru.push_back(b);
+                lru_pos[b] = std::prev(lru.end());
+                in_lru[b] = 1;
+            }
+        }
+    }
+    int64_t intern(int64_t parent, const int32_t* tokens) {
+        PrefixKey k{parent, std::vector<int32_t>(tokens, tokens + block_size)};
+        auto it = trie.find(k);
+        if (it != trie.end()) return it->second;
+        const int64_t node = static_cast<int64_t>(trie.size());
+        trie.emplace(std::move(k), node);
+        return node;
+    }
+    int64_t lookup(int64_t parent, const int32_t* tokens) const {
+        PrefixKey k{parent, std::vector<int32_t>(tokens, tokens + block_size)};
+        auto it = trie.find(k);
+        return it == trie.end() ? -1 : it->second;
     }
     int64_t slot(const Request& r, int64_t pos) const {
         return static_cast<int64_t>(r.table[pos / block_size]) * block_size + pos % block_size;
@@ -81,6 +170,9 @@ pa_status pa_alloc_create(int32_t num_blocks, int32_t block_size, const int32_t*
     a->num_blocks = num_blocks;
     a->block_size = block_size;
     a->refcount.assign(num_blocks, 0);
+    a->block_node.assign(num_blocks, -1);
+    a->lru_pos.resize(num_blocks);
+    a->in_lru.assign(num_blocks, 0);
     a->free_list.resize(num_blocks);
     if (init_free_order) {
         std::vector<char> seen(num_blocks, 0);
@@ -107,9 +199,10 @@ pa_status pa_alloc_allocate(pa_alloc* a, int64_t req, int32_t num_tokens) {
     if (num_tokens < 0) return fail(PA_ERR_INVALID_ARG, "pa_alloc_allocate: num_tokens=%d", num_tokens);
     if (a->reqs.count(req)) return fail(PA_ERR_EXISTS, "pa_alloc_allocate: request %lld exists", (long long)req);
     int64_t n = a->blocks_for(num_tokens);
-    if (n > static_cast<int64_t>(a->free_list.size())) {
+    if (n > a->available()) {
         a->oom_count += 1;
-        return fail(PA_ERR_OOM, "pa_alloc_allocate: need %lld blocks, %zu free", (long long)n, a->free_list.size());
+        return fail(PA_ERR_OOM, "pa_alloc_allocate: need %lld blocks, %lld available", (long long)n,
+                    (long long)a->available());
     }
     pa_alloc::Request r;
     r.table.reserve(n);
@@ -125,7 +218,7 @@ pa_status pa_alloc_append_token(pa_alloc* a, int64_t req, int64_t* slot_out) {
     if (it == a->reqs.end()) return fail(PA_ERR_NOT_FOUND, "pa_alloc_append_token: request %lld not found", (long long)req);
     pa_alloc::Request& r = it->second;
     if (r.len % a->block_size == 0) {
-        if (a->free_list.empty()) {
+        if (a->available() == 0) {
             a->oom_count += 1;
             return fail(PA_ERR_OOM, "pa_alloc_append_token: no free block");
         }
@@ -143,9 +236,10 @@ pa_status pa_alloc_append_tokens(pa_alloc* a, int64_t req, int32_t n, int64_t* s
     if (it == a->reqs.end()) return fail(PA_ERR_NOT_FOUND, "pa_alloc_append_tokens: request %lld not found", (long long)req);
     pa_alloc::Request& r = it->second;
     int64_t extra = a->blocks_for(static_cast<int64_t>(r.len) + n) - static_cast<int64_t>(r.table.size());
-    if (extra > static_cast<int64_t>(a->free_list.size())) {
+    if (extra > a->available()) {
         a->oom_count += 1;
-        return fail(PA_ERR_OOM, "pa_alloc_append_tokens: need %lld blocks, %zu free", (long long)extra, a->free_list.size());
+        return fail(PA_ERR_OOM, "pa_alloc_append_tokens: need %lld blocks, %lld available", (long long)extra,
+                    (long long)a->available());
     }
     for (int32_t i = 0; i < n; ++i) {
         if (r.len % a->block_size == 0) r.table.push_back(a->take());
@@ -175,9 +269,7 @@ pa_status pa_alloc_free(pa_alloc* a, int64_t req) {
     if (!a) return fail(PA_ERR_INVALID_ARG, "pa_alloc_free: NULL allocator");
     auto it = a->reqs.find(req);
     if (it == a->reqs.end()) return PA_OK;
-    for (int32_t b : it->second.table) {
-        if (--a->refcount[b] == 0) a->free_list.push_back(b);
-    }
+    a->release(it->second.table);
     a->reqs.erase(it);
     return PA_OK;
 }
@@ -267,6 +359,80 @@ pa_status pa_alloc_free_list(const pa_alloc* a, int32_t* out, int32_t cap, int32
     if (len_out) *len_out = n;
     if (cap < n || (n > 0 && !out)) return fail(PA_ERR_INVALID_ARG, "pa_alloc_free_list: capacity %d < %d", cap, n);
     if (n) std::memcpy(out, a->free_list.data(), sizeof(int32_t) * n);
+    return PA_OK;
+}
+
+pa_status pa_alloc_allocate_cached(pa_alloc* a, int64_t req, const int32_t* tokens, int32_t num_tokens,
+                                   int32_t* cached_tokens_out) {
+    if (!a) return fail(PA_ERR_INVALID_ARG, "pa_alloc_allocate_cached: NULL allocator");
+    if (num_tokens < 0 || (num_tokens > 0 && !tokens))
+        return fail(PA_ERR_INVALID_ARG, "pa_alloc_allocate_cached: num_tokens=%d", num_tokens);
+    if (a->reqs.count(req)) return fail(PA_ERR_EXISTS, "pa_alloc_allocate_cached: request %lld exists", (long long)req);
+    const int32_t bs = a->block_size;
+    const int64_t nfull = num_tokens / bs, nblocks = a->blocks_for(num_tokens);
+    // longest cached prefix of whole blocks
+    std::vector<int32_t> hits;
+    int64_t parent = -1;
+    for (int64_t i = 0; i < nfull; ++i) {
+        const int64_t node = a->lookup(parent, tokens + i * bs);
+        if (node < 0) break;
+        auto c = a->cache.find(node);
+        if (c == a->cache.end()) break;
+        hits.push_back(c->second);
+        parent = node;
+    }
+    int64_t parked_hits = 0;
+    for (int32_t b : hits) parked_hits += a->in_lru[b] ? 1 : 0;
+    const int64_t need = nblocks - static_cast<int64_t>(hits.size());
+    if (need > a->available() - parked_hits) {
+        a->oom_count += 1;
+        return fail(PA_ERR_OOM, "pa_alloc_allocate_cached: need %lld new blocks, %lld available", (long long)need,
+                    (long long)(a->available() - parked_hits));
+    }
+    pa_alloc::Request r;
+    r.table.reserve(nblocks);
+    for (int32_t b : hits) {
+        if (a->in_lru[b]) a->unpark(b);
+        a->refcount[b] += 1;
+        r.table.push_back(b);
+    }
+    for (int64_t i = 0; i < need; ++i) r.table.push_back(a->take());
+    // register the new full blocks under their prefix nodes
+    parent = -1;
+    for (int64_t i = 0; i < nfull; ++i) {
+        const int64_t node = a->intern(parent, tokens + i * bs);
+        if (i >= static_cast<int64_t>(hits.size()) && !a->cache.count(node)) {
+            a->cache.emplace(node, r.table[i]);
+            a->block_node[r.table[i]] = node;
+        }
+        parent = node;
+    }
+    r.len = num_tokens;
+    a->hit_blocks += static_cast<int64_t>(hits.size());
+    a->reqs.emplace(req, std::move(r));
+    if (cached_tokens_out) *cached_tokens_out = static_cast<int32_t>(hits.size()) * bs;
+    return PA_OK;
+}
+
+pa_status pa_alloc_cache_stats(const pa_alloc* a, pa_cache_stats_t* out) {
+    if (!a || !out) return fail(PA_ERR_INVALID_ARG, "pa_alloc_cache_stats: NULL argument");
+    pa_cache_stats_t s{};
+    s.cached_blocks = static_cast<int64_t>(a->cache.size());
+    s.evictable_blocks = static_cast<int64_t>(a->lru.size());
+    s.hit_blocks = a->hit_blocks;
+    s.evictions = a->evictions;
+    s.prefix_nodes = static_cast<int64_t>(a->trie.size());
+    *out = s;
+    return PA_OK;
+}
+
+pa_status pa_alloc_evictable_list(const pa_alloc* a, int32_t* out, int32_t cap, int32_t* len_out) {
+    if (!a) return fail(PA_ERR_INVALID_ARG, "pa_alloc_evictable_list: NULL allocator");
+    const int32_t n = static_cast<int32_t>(a->lru.size());
+    if (len_out) *len_out = n;
+    if (cap < n || (n > 0 && !out)) return fail(PA_ERR_INVALID_ARG, "pa_alloc_evictable_list: capacity %d < %d", cap, n);
+    int32_t i = 0;
+    for (int32_t b : a->lru) out[i++] = b;
     return PA_OK;
 }
 

@@ -219,3 +219,51 @@ def test_full_size_b256_sampled(cuda_ready):
 
 def test_full_size_long_context_sampled(cuda_ready):
     _sampled_full_size("longctx", [0, 3, 7])
+
+
+def test_decode_over_prefix_cached_blocks(cuda_ready):
+    """Requests sharing a system prompt through the allocator's prefix cache: later requests
+    write only their uncached tail, and decode reads the cached blocks written by the first."""
+    H, D, bs, N = 8, 128, 16, 40
+    rng = np.random.default_rng(21)
+    sys_tokens = rng.integers(0, 32000, 64).tolist()
+    sys_k = rng.standard_normal((64, H, D)).astype(np.float16)
+    sys_v = rng.standard_normal((64, H, D)).astype(np.float16)
+    alloc = pk.BlockAllocator(N, bs)
+    kc = torch.full((N, bs, H, D), float("nan"), dtype=torch.float16, device="cuda")
+    vc = torch.full_like(kc, float("nan"))
+    logical = {}
+    expect_cached = {"A": 0, "B": 64, "C": 64}
+    reqs = {"A": 0, "B": 1, "C": 2}
+    for name, n_suffix in (("A", 37), ("B", 50), ("C", 3)):
+        toks = sys_tokens + rng.integers(0, 32000, n_suffix).tolist()
+        st, cached = alloc.allocate_cached(reqs[name], toks)
+        assert st == pk.PA_OK and cached == expect_cached[name]
+        n = len(toks)
+        sk = rng.standard_normal((n_suffix, H, D)).astype(np.float16)
+        sv = rng.standard_normal((n_suffix, H, D)).astype(np.float16)
+        k_all, v_all = np.concatenate([sys_k, sk]), np.concatenate([sys_v, sv])
+        logical[name] = (k_all, v_all)
+        st, slots = alloc.slots(reqs[name], cached, n - cached)
+        pk.reshape_and_cache(torch.from_numpy(k_all[cached:]).cuda(), torch.from_numpy(v_all[cached:]).cuda(),
+                             kc, vc, torch.from_numpy(slots).cuda())
+        if name == "B":
+            alloc.free(reqs["A"])          # A leaves: its system blocks stay referenced by B
+            del logical["A"]
+    names = sorted(logical)
+    ids = [reqs[n] for n in names]
+    mb = 8
+    st, tables, lens = alloc.pack(ids, mb)
+    assert st == pk.PA_OK
+    q = rng.standard_normal((len(ids), H, D)).astype(np.float16)
+    out = torch.empty(len(ids), H, D, dtype=torch.float16, device="cuda")
+    ws = torch.empty(pk.decode_workspace_bytes(len(ids), H, D, mb, bs), dtype=torch.uint8, device="cuda")
+    pk.paged_attention_decode(out, torch.from_numpy(q).cuda(), kc, vc, torch.from_numpy(tables).cuda(),
+                              torch.from_numpy(lens).cuda(), 1 / np.sqrt(D), ws)
+    got = out.float().cpu().numpy()
+    for i, n in enumerate(names):
+        k_all, v_all = logical[n]
+        ref = oatt.softmax_attention(q[i][None], k_all, v_all, 1 / np.sqrt(D))[0]
+        assert np.abs(got[i] - ref).max() <= TOL
+    assert tables[0][:4].tolist() == tables[1][:4].tolist()      # B and C share the 4 prompt blocks
+    assert alloc.cache_stats()["hit_blocks"] == 8

@@ -1,0 +1,114 @@
+"""Automatic prefix caching: the oracle against a hand-traced golden log and the page's
+shared system-prompt example, then the C++ allocator against the oracle, bit for bit, on
+random logs of prefix-sharing requests (no GPU)."""
+import numpy as np
+import pytest
+from hypothesis import given, settings
+from hypothesis import strategies as st
+
+import paged_kv_cache_411_b200 as pk
+from conftest import golden
+from oracle import block_manager as obm
+from oracle.prefix_cache import PrefixCachingBlockManager
+
+_NAMES = {pk.PA_OK: obm.OK, pk.PA_ERR_OOM: obm.OOM, pk.PA_ERR_NOT_FOUND: obm.NOT_FOUND,
+          pk.PA_ERR_EXISTS: obm.EXISTS, pk.PA_ERR_INVALID_ARG: obm.INVALID_ARG}
+
+
+def test_oracle_follows_hand_trace():
+    g = golden("prefix_cache_trace.json")
+    bm = PrefixCachingBlockManager(g["num_blocks"], g["block_size"])
+    for op in g["ops"]:
+        kind = op[0]
+        if kind == "allocate_cached":
+            st_, cached = bm.allocate_cached(op[1], op[2])
+            assert (st_, cached) == (op[3], op[4]), op
+            if op[5] is not None:
+                assert bm.block_tables[op[1]] == op[5], op
+        elif kind == "allocate":
+            assert bm.allocate(op[1], op[2]) == op[3]
+            assert bm.block_tables[op[1]] == op[4]
+        elif kind == "free":
+            assert bm.free(op[1]) == op[2]
+        elif kind == "check_lru":
+            assert list(bm.lru) == op[1], op
+        elif kind == "check_free":
+            assert bm.free_blocks == op[1], op
+        elif kind == "check_refcount":
+            assert bm.refcount == op[1], op
+
+
+def test_shared_system_prompt_is_stored_once():
+    """The page's figure: a 3-block system prompt shared by two requests with 2 private blocks
+    each occupies 7 blocks; the second request finds all 3 prompt blocks in the cache."""
+    bs = 16
+    rng = np.random.default_rng(0)
+    system = rng.integers(0, 32000, 3 * bs).tolist()
+    q1 = rng.integers(0, 32000, 20).tolist()
+    q2 = rng.integers(0, 32000, 25).tolist()
+    bm = PrefixCachingBlockManager(32, bs)
+    assert bm.allocate_cached(1, system + q1) == (obm.OK, 0)
+    assert bm.allocate_cached(2, system + q2) == (obm.OK, 3 * bs)
+    assert bm.block_tables[1][:3] == bm.block_tables[2][:3]
+    assert not set(bm.block_tables[1][3:]) & set(bm.block_tables[2][3:])
+    assert bm.stats()["num_used"] == 7 and bm.cache_stats()["hit_blocks"] == 3
+    assert all(bm.refcount[b] == 2 for b in bm.block_tables[1][:3])
+    # a different prompt shares nothing; the same prompt after both left is still cached
+    bm.free(1)
+    bm.free(2)
+    assert bm.allocate_cached(3, rng.integers(0, 32000, 48).tolist()) == (obm.OK, 0)
+    assert bm.allocate_cached(4, system + [7]) == (obm.OK, 3 * bs)
+    # identical block content after a different prefix is a different block
+    other = rng.integers(0, 32000, bs).tolist()
+    assert bm.allocate_cached(5, other + system[bs:2 * bs]) == (obm.OK, 0)
+
+
+def _replay(N, bs, log, vocab):
+    ca = pk.BlockAllocator(N, bs)
+    om = PrefixCachingBlockManager(N, bs)
+    for kind, a, b, fam, n in log:
+        if kind == 0:
+            base = [fam * 1000 + i for i in range(n)]
+            toks = base[: n - (b % 3)] + [(vocab * b + i) % 7 for i in range(b % 3)]
+            st, cached = ca.allocate_cached(a, toks)
+            ost, ocached = om.allocate_cached(a, toks)
+            assert (_NAMES[st], cached) == (ost, ocached)
+        elif kind == 1:
+            assert _NAMES[ca.allocate(a, n)] == om.allocate(a, n)
+        elif kind == 2:
+            st, slot = ca.append_token(a)
+            ost, oslot = om.append_token(a)
+            assert _NAMES[st] == ost and slot == oslot
+        elif kind == 3:
+            p = min(n, om.seq_lens.get(a, 0))
+            assert _NAMES[ca.fork(a, b, p)] == om.fork(a, b, p)
+        else:
+            assert _NAMES[ca.free(a)] == om.free(a)
+        assert ca.free_list().tolist() == om.free_blocks
+        assert ca.evictable_list().tolist() == list(om.lru)
+    for r in range(6):
+        st, t = ca.get_block_table(r)
+        assert t.tolist() == om.get_block_table(r)[1]
+    assert [ca.refcount(b)[1] for b in range(N)] == om.refcount
+    assert ca.cache_stats() == om.cache_stats()
+    s1, s2 = ca.stats(), om.stats()
+    assert all(s1[k] == s2[k] for k in s2)
+
+
+ops = st.lists(st.tuples(st.integers(0, 4), st.integers(0, 5), st.integers(0, 5), st.integers(0, 2),
+                         st.integers(0, 40)), min_size=1, max_size=120)
+
+
+@settings(max_examples=300, deadline=None)
+@given(st.integers(1, 24), st.sampled_from([1, 2, 4, 8]), st.integers(1, 5), ops)
+def test_cpp_prefix_cache_matches_oracle(N, bs, vocab, log):
+    _replay(N, bs, log, vocab)
+
+
+def test_prefix_cache_errors():
+    ca = pk.BlockAllocator(4, 2)
+    assert ca.allocate_cached(1, [1, 2, 3]) == (pk.PA_OK, 0)
+    assert ca.allocate_cached(1, [1, 2]) == (pk.PA_ERR_EXISTS, 0)
+    assert ca.allocate_cached(2, [1, 2, 9, 9, 9, 9, 9]) == (pk.PA_ERR_OOM, 0)
+    assert ca.stats()["oom_count"] == 1 and ca.cache_stats()["cached_blocks"] == 1
+    assert ca.allocate_cached(3, []) == (pk.PA_OK, 0)
