@@ -202,6 +202,41 @@ pa_status pa_alloc_cache_stats(const pa_alloc* a, pa_cache_stats_t* out);
  * eviction takes out[0]).  Errors: INVALID_ARG (cap < length; *len_out set). */
 pa_status pa_alloc_evictable_list(const pa_alloc* a, int32_t* out, int32_t cap, int32_t* len_out);
 
+/* ---- swap between the GPU pool and a host pool ([CB-PA] §4.4 Swap: CPU
+ * offload, one block manager per pool; §5.4 preemption by swapping) ---------
+ *
+ * Pools are the K and V pool tensors of two allocators with the same
+ * block_size; one block of one pool is `block_bytes` bytes (block_size *
+ * num_heads * head_dim * 2 for fp16).  Memory may be device memory or pinned
+ * host memory on either side (copies use cudaMemcpyDefault).  Copies are
+ * asynchronous on `stream`; the caller keeps the buffers alive until they
+ * complete. */
+
+/* Copy K and V blocks: for each pair i, block mapping[2i] of (src_k, src_v)
+ * to block mapping[2i+1] of (dst_k, dst_v) (host int64 mapping[num_pairs][2]).
+ * Runs of consecutive pairs become one cudaMemcpyAsync each, in list order.
+ * num_pairs == 0 or block_bytes == 0 copies nothing.
+ * Errors: INVALID_ARG (pair outside [0, src/dst_num_blocks)), CUDA. */
+pa_status pa_swap_blocks(const void* src_k, const void* src_v, void* dst_k, void* dst_v,
+                         const int64_t* mapping, int32_t num_pairs, int64_t block_bytes,
+                         int32_t src_num_blocks, int32_t dst_num_blocks, void* stream);
+
+/* Swap `req` out of the GPU pool: allocate it in `cpu` with its seq_len,
+ * copy its blocks GPU -> host, free it in `gpu` (its GPU blocks may be
+ * reused by work ordered after the copy on `stream`).  Shared blocks are
+ * copied and only lose this request's reference.  block_bytes == 0 does the
+ * bookkeeping alone.
+ * Errors: NOT_FOUND (req not in gpu), EXISTS (req already in cpu), OOM (cpu
+ * pool full; nothing changes), INVALID_ARG (block sizes differ), CUDA (the
+ * cpu allocation is rolled back). */
+pa_status pa_alloc_swap_out(pa_alloc* gpu, pa_alloc* cpu, int64_t req, const void* gpu_k,
+                            const void* gpu_v, void* cpu_k, void* cpu_v, int64_t block_bytes,
+                            void* stream);
+/* The reverse move: allocate `req` in `gpu`, copy host -> GPU, free it in `cpu`.
+ * Errors: as pa_alloc_swap_out with the pools exchanged. */
+pa_status pa_alloc_swap_in(pa_alloc* gpu, pa_alloc* cpu, int64_t req, void* gpu_k, void* gpu_v,
+                           const void* cpu_k, const void* cpu_v, int64_t block_bytes, void* stream);
+
 /* ---- device kernels -------------------------------------------------------- */
 
 /* reshape_and_cache: write the step's new K/V rows into the pool.

@@ -23,7 +23,8 @@ from ._lib import (PA_DEVCHK_BLOCK_ID, PA_DEVCHK_QUERY_RANGE, PA_DEVCHK_SEQ_LEN,
 
 __all__ = [
     "BlockAllocator", "reshape_and_cache", "paged_attention_decode", "paged_attention_prefill_chunk",
-    "decode_workspace_bytes", "paged_attention_decode_noalloc", "PagedKVError", "lib", "STATUS_NAMES", "PA_OK", "PA_ERR_INVALID_ARG",
+    "decode_workspace_bytes", "paged_attention_decode_noalloc", "swap_blocks", "swap_out", "swap_in",
+    "PagedKVError", "lib", "STATUS_NAMES", "PA_OK", "PA_ERR_INVALID_ARG",
     "PA_ERR_OOM", "PA_ERR_NOT_FOUND", "PA_ERR_EXISTS", "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA",
     "PA_ERR_DEVICE_CHECK", "PA_DEVCHK_BLOCK_ID", "PA_DEVCHK_SLOT", "PA_DEVCHK_SEQ_LEN",
     "PA_DEVCHK_QUERY_RANGE", "PA_DEVCHK_TIMEOUT",
@@ -144,6 +145,44 @@ class BlockAllocator:
         out = np.empty(n.value, dtype=np.int32)
         check(lib().pa_alloc_evictable_list(self._h, _i32p(out), n.value, byref(n)))
         return out
+
+
+# ------------------------------------------------------------------ swapping
+def _ptr_any(t):
+    if t is None:
+        return None
+    return c_void_p(t.data_ptr() if hasattr(t, "data_ptr") else int(t))
+
+
+def _stream_handle(stream):
+    if stream is None:
+        try:
+            import torch
+            if torch.cuda.is_available():
+                return c_void_p(torch.cuda.current_stream().cuda_stream)
+        except ImportError:
+            pass
+        return None
+    return c_void_p(stream.cuda_stream)
+
+
+def swap_blocks(src_k, src_v, dst_k, dst_v, mapping, block_bytes, src_num_blocks, dst_num_blocks, stream=None):
+    """pa_swap_blocks: mapping is an int64 [n, 2] host array of (source block, destination block)."""
+    m = np.ascontiguousarray(mapping, dtype=np.int64).reshape(-1, 2)
+    check(lib().pa_swap_blocks(_ptr_any(src_k), _ptr_any(src_v), _ptr_any(dst_k), _ptr_any(dst_v), _i64p(m),
+                               len(m), int(block_bytes), src_num_blocks, dst_num_blocks, _stream_handle(stream)))
+
+
+def swap_out(gpu_alloc, cpu_alloc, req, gpu_k, gpu_v, cpu_k, cpu_v, block_bytes, stream=None) -> int:
+    """pa_alloc_swap_out; returns the status (PA_ERR_OOM when the host pool is full)."""
+    return lib().pa_alloc_swap_out(gpu_alloc._h, cpu_alloc._h, req, _ptr_any(gpu_k), _ptr_any(gpu_v),
+                                   _ptr_any(cpu_k), _ptr_any(cpu_v), int(block_bytes), _stream_handle(stream))
+
+
+def swap_in(gpu_alloc, cpu_alloc, req, gpu_k, gpu_v, cpu_k, cpu_v, block_bytes, stream=None) -> int:
+    """pa_alloc_swap_in; returns the status (PA_ERR_OOM when the GPU pool is full)."""
+    return lib().pa_alloc_swap_in(gpu_alloc._h, cpu_alloc._h, req, _ptr_any(gpu_k), _ptr_any(gpu_v),
+                                  _ptr_any(cpu_k), _ptr_any(cpu_v), int(block_bytes), _stream_handle(stream))
 
 
 # ------------------------------------------------------------------ kernels

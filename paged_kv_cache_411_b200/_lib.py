@@ -87,6 +87,9 @@ SIGNATURES = {
     "pa_alloc_allocate_cached": (c_int32, [_P, c_int64, _I32P, c_int32, _I32P]),
     "pa_alloc_cache_stats": (c_int32, [_P, POINTER(CacheStats)]),
     "pa_alloc_evictable_list": (c_int32, [_P, _I32P, c_int32, _I32P]),
+    "pa_swap_blocks": (c_int32, [_P, _P, _P, _P, _I64P, c_int32, c_int64, c_int32, c_int32, _P]),
+    "pa_alloc_swap_out": (c_int32, [_P, _P, c_int64, _P, _P, _P, _P, c_int64, _P]),
+    "pa_alloc_swap_in": (c_int32, [_P, _P, c_int64, _P, _P, _P, _P, c_int64, _P]),
     "pa_reshape_and_cache": (c_int32, [_P, _P, _P, _P, _P, c_int32, c_int32, c_int32, c_int32, c_int32, _P, _P]),
     "pa_decode_workspace_bytes": (c_size_t, [c_int32, c_int32, c_int32, c_int32, c_int32]),
     "pa_paged_attention_decode": (c_int32, [_P, _P, _P, _P, _P, _P, c_int32, c_int32, c_int32, c_int32, c_int32,

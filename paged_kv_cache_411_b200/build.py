@@ -27,6 +27,7 @@ SOURCES = [
     "block_allocator.cpp",
     "capi.cpp",
     "runtime.cpp",
+    "swap.cpp",
     "reshape_and_cache.cu",
     "decode.cu",
     "decode_noalloc.cu",
