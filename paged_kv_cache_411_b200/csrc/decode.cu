@@ -30,9 +30,14 @@
 //     transposing warp-shuffle reduction, and P.V accumulates in registers.
 //     The warps sharing a head merge their (max, sum, acc) through shared
 //     memory at the end of the item; single-partition sequences are written
-//     straight to `out`, others write an fp32 partial.
-//  3. combine kernel: merges partials with the exact log-sum-exp rule
-//     m* = max m_i, l* = sum l_i 2^(m_i - m*), o* = sum acc_i 2^(m_i - m*) / l*.
+//     straight to `out`, others write an fp32 partial and take a ticket for
+//     their (sequence, head): the warp that takes the last ticket merges all
+//     partitions with the exact log-sum-exp rule
+//     m* = max m_i, l* = sum l_i 2^(m_i - m*), o* = sum acc_i 2^(m_i - m*) / l*
+//     and writes the output, so no separate combine launch is needed.
+//  The streaming kernel is launched as a programmatic dependent of the plan
+//  kernel: its CTAs become resident and set up their barriers and TMA
+//  descriptors while the plan runs, and wait for it with griddepcontrol.
 //
 // The combine order is the partition order and the in-item merge order is
 // fixed, so the result does not depend on physical block placement (bitwise)
@@ -59,9 +64,9 @@ constexpr int kLast = 1 << 9;
 constexpr int kSingle = 1 << 10;
 constexpr int kTerminate = 1 << 11;
 
-// Item record: x = seq, y = first token, z = tokens, w = (partition << 9) | (single << 8) | head group.
+// Item record: x = seq, y = first token, z = tokens | (head group << 10), w = partition | (partitions << 16).
 struct WsLayout {
-    size_t hdr, n_splits, items, part_ml, part_acc, total;
+    size_t hdr, n_splits, items, part_ml, part_acc, tickets, total;
     int32_t max_splits;
 };
 
@@ -78,6 +83,7 @@ inline WsLayout ws_layout(int32_t S, int32_t H, int32_t D, int32_t max_blocks, i
     w.items = off;      off = align256(off + sizeof(int4) * pairs * H);
     w.part_ml = off;    off = align256(off + sizeof(float2) * pairs * H);
     w.part_acc = off;   off = align256(off + sizeof(float) * pairs * H * D);
+    w.tickets = off;    off = align256(off + sizeof(int32_t) * static_cast<size_t>(S) * H);
     w.total = off;
     return w;
 }
@@ -93,9 +99,13 @@ struct DecodeParams {
     int4* items;
     float2* part_ml;
     float* part_acc;
+    int32_t* tickets;                   // [S][H] partitions merged so far (zeroed by the plan)
     int32_t max_splits;
     int32_t* err_flag;
 };
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 template <int D, int HG>
 struct Cfg {
@@ -185,7 +195,8 @@ __device__ __forceinline__ float reduce_scores(float (&v)[NV], int lane) {
 
 // ------------------------------------------------------------------ plan ----
 __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeParams p, int32_t hg_count,
-                                                           int32_t target_items, int32_t max_split) {
+                                                           int32_t target_items, int32_t max_split,
+                                                           int32_t head_dim) {
     constexpr int kNC = 4;
     const int cand[kNC] = {512, 256, 128, 64};
     __shared__ long long red[kNC][32];
@@ -193,6 +204,8 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeParams p, int32
     __shared__ long long s_scan[2][32];
     __shared__ long long s_tot[2];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+    pdl_wait();                       // inputs may come from the kernel before us on the stream
+    pdl_launch_dependents();          // let the streaming kernel's CTAs set up meanwhile
 
     long long cnt[kNC] = {0, 0, 0, 0};
     for (int s = tid; s < p.S; s += blockDim.x) {
@@ -259,14 +272,19 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeParams p, int32
         const int nfull = len / split, tail = len % split;
         const int nsp = nfull + (tail != 0);
         p.n_splits[s] = nsp;
-        const int single = nsp == 1 ? (1 << 8) : 0;
         for (int k = 0; k < nfull; ++k, ++off_f)
             for (int g = 0; g < hg_count; ++g)
-                p.items[off_f * hg_count + g] = make_int4(s, k * split, split, (k << 9) | single | g);
+                p.items[off_f * hg_count + g] = make_int4(s, k * split, split | (g << 10), k | (nsp << 16));
         if (tail) {
             for (int g = 0; g < hg_count; ++g)
-                p.items[off_p * hg_count + g] = make_int4(s, nfull * split, tail, (nfull << 9) | single | g);
+                p.items[off_p * hg_count + g] = make_int4(s, nfull * split, tail | (g << 10), nfull | (nsp << 16));
             ++off_p;
+        }
+        if (nsp > 1)
+            for (int h = 0; h < p.H; ++h) p.tickets[static_cast<int64_t>(s) * p.H + h] = 0;
+        if (nsp == 0) {                 // empty sequence: zeros
+            uint4* o = reinterpret_cast<uint4*>(p.out + static_cast<int64_t>(s) * p.H * head_dim);
+            for (int i = 0; i < p.H * head_dim / 8; ++i) o[i] = make_uint4(0, 0, 0, 0);
         }
     }
     if (tid == 0) {
@@ -274,6 +292,33 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeParams p, int32
         p.hdr[1] = static_cast<int32_t>((s_tot[0] + s_tot[1]) * hg_count);
         p.hdr[2] = split;
     }
+}
+
+// Merge the nsp fp32 partials of (seq, head) with the log-sum-exp rule and write the fp16 output.
+// Called by one warp, after every partial of the pair is visible (ticket protocol); reads bypass L1.
+template <int D>
+__device__ __forceinline__ void combine_head(const DecodeParams& p, int seq, int head, int nsp, int lane) {
+    constexpr int VEC = D / 32;
+    const int64_t base = static_cast<int64_t>(seq) * p.max_splits * p.H + head;
+    float M = -INFINITY;
+    for (int i = lane; i < nsp; i += 32) M = fmaxf(M, __ldcg(&p.part_ml[base + static_cast<int64_t>(i) * p.H]).x);
+    for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float L = 0.f, acc[VEC];
+#pragma unroll
+    for (int k = 0; k < VEC; ++k) acc[k] = 0.f;
+    for (int i = 0; i < nsp; ++i) {
+        const int64_t pi = base + static_cast<int64_t>(i) * p.H;
+        const float2 ml = __ldcg(&p.part_ml[pi]);
+        const float w = exp2f(ml.x - M);
+        L = fmaf(ml.y, w, L);
+        const float* a = p.part_acc + pi * D + lane * VEC;
+#pragma unroll
+        for (int k = 0; k < VEC; ++k) acc[k] = fmaf(__ldcg(a + k), w, acc[k]);
+    }
+    const float r = 1.f / L;
+    __half* o = p.out + (static_cast<int64_t>(seq) * p.H + head) * D + lane * VEC;
+#pragma unroll
+    for (int k = 0; k < VEC; k += 2) *reinterpret_cast<uint32_t*>(o + k) = f2_to_h2(acc[k] * r, acc[k + 1] * r);
 }
 
 // ------------------------------------------------------------------ main ----
@@ -308,6 +353,7 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         mbar_init_fence();
     }
     __syncthreads();
+    pdl_wait();                       // the plan (and everything before it) has completed
 
     const int n_items = p.hdr[1];
 
@@ -332,8 +378,9 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         idx = __shfl_sync(0xffffffffu, idx, 0);
         int4 rec = idx < n_items ? p.items[idx] : make_int4(-1, 0, 0, 0);
         while (rec.x >= 0 && ok) {
-            const int seq = rec.x, tok0 = rec.y, ntok_item = rec.z;
-            const int hg = rec.w & 0xff, single = rec.w & (1 << 8), part = rec.w >> 9;
+            const int seq = rec.x, tok0 = rec.y, ntok_item = rec.z & 1023, hg = rec.z >> 10;
+            const int part = rec.w & 0xffff, nsp = rec.w >> 16;
+            const int single = nsp == 1;
             int nidx = 0;
             if (lane == 0) nidx = atomicAdd(&p.hdr[0], 1);       // next item, in flight meanwhile
             const int blk0 = tok0 / bs;
@@ -358,7 +405,7 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                     int flags = ntok;
                     if (st == 0) flags |= kFirst;
                     if (st == nst - 1) flags |= kLast | (single ? kSingle : 0);
-                    info[stage] = make_int4(seq, part, hg, flags);
+                    info[stage] = make_int4(seq, part | (nsp << 16), hg, flags);
                     const int nbox = (bs >= kStageTok) ? 1 : (ntok + box_tok - 1) / box_tok;
                     const uint32_t kv_bytes = nbox * box_bytes;
                     uint8_t* dk = tile_k + size_t(stage) * C::kTileBytes;
@@ -515,7 +562,7 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                     a8[4] = fmaf(y.x, wj, a8[4]); a8[5] = fmaf(y.y, wj, a8[5]);
                     a8[6] = fmaf(y.z, wj, a8[6]); a8[7] = fmaf(y.w, wj, a8[7]);
                 }
-                const int seq = inf.x, part = inf.y, head = inf.z * HG + hh;
+                const int seq = inf.x, part = inf.y & 0xffff, nsp = inf.y >> 16, head = inf.z * HG + hh;
                 if (flags & kSingle) {
                     if (tq == 0) {
                         const float r = 1.f / L;
@@ -534,49 +581,22 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                         *reinterpret_cast<float4*>(dst + 4) = make_float4(a8[4], a8[5], a8[6], a8[7]);
                     }
                     if (lane == 0) p.part_ml[pi] = make_float2(M, L);
+                    // Publish the partial, then take a ticket; the last partition merges them all.
+                    __threadfence();
+                    __syncwarp();
+                    int ticket = 0;
+                    if (lane == 0) ticket = atomicAdd(&p.tickets[static_cast<int64_t>(seq) * p.H + head], 1);
+                    ticket = __shfl_sync(0xffffffffu, ticket, 0);
+                    if (ticket == nsp - 1) {
+                        __threadfence();
+                        combine_head<D>(p, seq, head, nsp, lane);
+                    }
                 }
             }
         }
         if (*abort_flag) break;
         if (++stage == C::kStages) { stage = 0; phase ^= 1; }
     }
-}
-
-// --------------------------------------------------------------- combine ----
-template <int D>
-__global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
-    constexpr int VEC = D / 32;
-    const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (gw >= p.S * p.H) return;
-    const int s = gw / p.H, h = gw % p.H;
-    const int n = p.n_splits[s];
-    if (n == 1) return;
-    __half* o = p.out + static_cast<int64_t>(gw) * D + lane * VEC;
-    if (n == 0) {
-#pragma unroll
-        for (int k = 0; k < VEC; k += 2) *reinterpret_cast<uint32_t*>(o + k) = f2_to_h2(0.f, 0.f);
-        return;
-    }
-    const int64_t base = static_cast<int64_t>(s) * p.max_splits * p.H + h;
-    float M = -INFINITY;
-    for (int i = lane; i < n; i += 32) M = fmaxf(M, p.part_ml[base + static_cast<int64_t>(i) * p.H].x);
-    for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float L = 0.f, acc[VEC];
-#pragma unroll
-    for (int k = 0; k < VEC; ++k) acc[k] = 0.f;
-    for (int i = 0; i < n; ++i) {
-        const int64_t pi = base + static_cast<int64_t>(i) * p.H;
-        const float2 ml = p.part_ml[pi];
-        const float w = exp2f(ml.x - M);
-        L = fmaf(ml.y, w, L);
-        const float* a = p.part_acc + pi * D + lane * VEC;
-#pragma unroll
-        for (int k = 0; k < VEC; ++k) acc[k] = fmaf(a[k], w, acc[k]);
-    }
-    const float r = 1.f / L;
-#pragma unroll
-    for (int k = 0; k < VEC; k += 2) *reinterpret_cast<uint32_t*>(o + k) = f2_to_h2(acc[k] * r, acc[k + 1] * r);
 }
 
 template <int D, int HG>
@@ -590,8 +610,17 @@ cudaError_t run_main(const CUtensorMap& tk, const CUtensorMap& tv, const CUtenso
                                         static_cast<int>(C::kSmemBytes));
     });
     if (attr_err != cudaSuccess) return attr_err;
-    decode_main_kernel<D, HG><<<grid, kThreads, C::kSmemBytes, stream>>>(tk, tv, tq, p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_main_kernel<D, HG>, tk, tv, tq, p);
 }
 
 }  // namespace
@@ -631,6 +660,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream, const char**
     p.items = reinterpret_cast<int4*>(ws + w.items);
     p.part_ml = reinterpret_cast<float2*>(ws + w.part_ml);
     p.part_acc = reinterpret_cast<float*>(ws + w.part_acc);
+    p.tickets = reinterpret_cast<int32_t*>(ws + w.tickets);
     p.max_splits = w.max_splits;
     p.err_flag = a.err_flag;
     if (a.num_seqs == 0) return cudaSuccess;
@@ -646,9 +676,20 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream, const char**
 
     const int sms = device_sm_count();
     const int max_split = a.block_size >= 16 ? 512 : 32 * a.block_size;
-    decode_plan_kernel<<<1, 1024, 0, stream>>>(p, a.num_heads / HG, 8 * sms, max_split);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    cudaError_t e;
+    {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(1);
+        cfg.blockDim = dim3(1024);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, decode_plan_kernel, p, a.num_heads / HG, 8 * sms, max_split, a.head_dim);
+        if (e != cudaSuccess) return e;
+    }
     if (a.head_dim == 128) {
         if (HG == 8) e = run_main<128, 8>(tk, tv, tq, p, sms, stream);
         else if (HG == 4) e = run_main<128, 4>(tk, tv, tq, p, sms, stream);
@@ -657,11 +698,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream, const char**
         if (HG == 8) e = run_main<64, 8>(tk, tv, tq, p, sms, stream);
         else e = run_main<64, 4>(tk, tv, tq, p, sms, stream);
     }
-    if (e != cudaSuccess) return e;
-    const int warps = a.num_seqs * a.num_heads;
-    if (a.head_dim == 128) decode_combine_kernel<128><<<(warps + 7) / 8, 256, 0, stream>>>(p);
-    else decode_combine_kernel<64><<<(warps + 7) / 8, 256, 0, stream>>>(p);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace pagedkv
