@@ -237,6 +237,84 @@ pa_status pa_alloc_swap_out(pa_alloc* gpu, pa_alloc* cpu, int64_t req, const voi
 pa_status pa_alloc_swap_in(pa_alloc* gpu, pa_alloc* cpu, int64_t req, void* gpu_k, void* gpu_v,
                            const void* cpu_k, const void* cpu_v, int64_t block_bytes, void* stream);
 
+/* ---- continuous-batching step driver ([CB-PA] §2.2 iteration-level
+ * scheduler and mixed prefill/decode batch, §4.3 chunked prefill, §5.3
+ * watermark admission, §5.4 preemption by recomputation; [DB] §4.4 loop) -----
+ *
+ * One step: (1) free requests that produced their last token; (2) while the
+ * running decodes need more new blocks than are available, preempt the most
+ * recently admitted running request (blocks freed, back to the FRONT of the
+ * waiting queue, it will recompute its prompt plus its generated tokens);
+ * (3) admit waiting requests in arrival order while fewer than max_num_seqs
+ * run and the blocks of the whole prefill + the decodes' needs +
+ * watermark_blocks are available; (4) every fully prefilled request decodes
+ * one token, then requests still prefilling get chunks, in running order,
+ * from a budget of max_num_tokens prefill tokens (whole prompts only when
+ * chunked_prefill is 0; a chunk without blocks waits).  The allocator is
+ * borrowed (it must outlive the scheduler) and is driven only through its
+ * public calls.  Not thread-safe. */
+
+typedef struct pa_sched pa_sched;
+
+typedef struct {
+    int32_t max_num_seqs;       /* cap on running requests (= on a step's batch)      */
+    int32_t max_num_tokens;     /* prefill-token budget of one step                   */
+    int32_t chunked_prefill;    /* 1: split prompts into chunks; 0: whole prompts     */
+    int32_t watermark_blocks;   /* blocks admission leaves free                       */
+} pa_sched_config_t;
+
+typedef struct {
+    int64_t step;               /* index of this step                                 */
+    int32_t num_prefill;        /* prefill entries                                    */
+    int32_t num_decode;         /* decode entries                                     */
+    int32_t num_tokens;         /* rows of the step's slot mapping                    */
+    int32_t num_admitted;
+    int32_t num_preempted;
+    int32_t num_finished;       /* requests freed at the start of this step           */
+} pa_step_info_t;
+
+typedef struct {
+    int32_t state;              /* 0 waiting, 1 running, 2 finished                   */
+    int32_t prompt_len;
+    int32_t max_new_tokens;
+    int32_t prefilled;          /* tokens of the current prefill already cached       */
+    int32_t to_prefill;         /* prompt (+ generated tokens after a preemption)     */
+    int32_t generated;
+    int32_t preemptions;
+    int32_t pad_;
+    int64_t first_token_step;   /* step that emitted its first token, -1 if none      */
+    int64_t finish_step;        /* step that emitted its last token, -1 if none       */
+} pa_request_info_t;
+
+typedef struct {
+    int64_t steps, waiting, running, finished, preemptions, prefill_tokens, decode_tokens;
+} pa_sched_stats_t;
+
+/* Errors: INVALID_ARG (NULL, non-positive caps, negative watermark). */
+pa_status pa_sched_create(pa_alloc* alloc, const pa_sched_config_t* cfg, pa_sched** out);
+void pa_sched_destroy(pa_sched* s);
+/* Queue a request (arrival order = call order).  Errors: INVALID_ARG
+ * (prompt_len or max_new_tokens <= 0), EXISTS (id known to the scheduler or
+ * holding blocks in the allocator). */
+pa_status pa_sched_add_request(pa_sched* s, int64_t req, int32_t prompt_len, int32_t max_new_tokens);
+/* Schedule one step (host buffers, any may be NULL): prefill_reqs /
+ * prefill_ctx (tokens already cached) / prefill_len (chunk) and decode_reqs /
+ * decode_seq_lens (including the new token) hold up to max_num_seqs entries;
+ * slot_mapping up to max_num_tokens + max_num_seqs rows: the prefill chunks'
+ * rows in prefill order, then one row per decode.  A request's prefill rows
+ * are its positions prefill_ctx .. prefill_ctx + prefill_len - 1.
+ * Errors: INVALID_ARG (previous step not completed). */
+pa_status pa_sched_step(pa_sched* s, pa_step_info_t* info, int64_t* prefill_reqs, int32_t* prefill_ctx,
+                        int32_t* prefill_len, int64_t* decode_reqs, int32_t* decode_seq_lens,
+                        int64_t* slot_mapping);
+/* Apply the scheduled step after its kernels ran: chunks become cached; a
+ * request whose prefill completed, and each decode, emits one token; a request
+ * that emitted max_new_tokens finishes (freed at the next step).
+ * Errors: INVALID_ARG (no open step). */
+pa_status pa_sched_complete(pa_sched* s);
+pa_status pa_sched_request_info(const pa_sched* s, int64_t req, pa_request_info_t* out);
+pa_status pa_sched_stats(const pa_sched* s, pa_sched_stats_t* out);
+
 /* ---- device kernels -------------------------------------------------------- */
 
 /* reshape_and_cache: write the step's new K/V rows into the pool.

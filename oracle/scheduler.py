@@ -1,0 +1,158 @@
+"""Oracle continuous-batching scheduler (test infrastructure only).
+
+Page "LLM 推理引擎 Continuous Batching 与 PagedAttention": §2.2
+(``ContinuousBatchingScheduler.step``: free finished requests, admit waiting
+ones while ``_can_allocate``, build a batch with prefill first under
+``max_num_tokens`` and one token per decode), §4.3 (chunked prefill), §5.3
+(admission keeps a block watermark), §5.4 (preemption: the newest running
+request goes back to the front of the waiting queue and its blocks are freed;
+"recompute" redoes its tokens).  Chapter "动态批处理算法" §4.4 gives the same
+loop.  Readings where the sketch leaves a step open:
+
+* preemption happens before admission, only as far as the running decodes
+  need new blocks that are not available (the sketch preempts while no block is
+  free); a preempted request recomputes its prompt plus the tokens it
+  generated;
+* ``_can_allocate`` admits a request when the blocks of its whole prefill, the
+  decodes' needs and the watermark are available;
+* decodes get their token before prefills get chunks (so admission can never
+  starve them of blocks); prefill chunks go in running order, at most the
+  remaining token budget each (whole prompts only without chunking); a chunk
+  that cannot get its blocks waits; the step's slot mapping lists the prefill
+  rows, then the decode rows;
+* finishing: a request emits a token when its prefill completes and at each
+  decode; at ``max_new_tokens`` it finishes and is freed at the next step.
+"""
+from __future__ import annotations
+
+from collections import deque
+
+from .block_manager import OK, OOM
+from .sizes import blocks_needed
+
+WAITING, RUNNING, FINISHED = 0, 1, 2
+
+
+class _Req:
+    def __init__(self, prompt_len, max_new):
+        self.prompt_len = prompt_len
+        self.max_new = max_new
+        self.to_prefill = prompt_len
+        self.prefilled = 0
+        self.generated = 0
+        self.state = WAITING
+        self.first_token_step = -1
+        self.finish_step = -1
+        self.preemptions = 0
+
+
+class Scheduler:
+    def __init__(self, bm, max_num_seqs, max_num_tokens, chunked_prefill=True, watermark_blocks=0):
+        self.bm = bm
+        self.max_num_seqs = max_num_seqs
+        self.max_num_tokens = max_num_tokens
+        self.chunked = bool(chunked_prefill)
+        self.watermark = watermark_blocks
+        self.reqs: dict = {}
+        self.waiting: deque = deque()
+        self.running: list = []
+        self.steps = 0
+        self.last_prefill: list = []
+        self.last_decode: list = []
+
+    def add_request(self, req, prompt_len, max_new):
+        self.reqs[req] = _Req(prompt_len, max_new)
+        self.waiting.append(req)
+        return OK
+
+    def _decoding(self, q):
+        return q.state == RUNNING and q.prefilled == q.to_prefill and q.generated < q.max_new
+
+    def _need(self):
+        bs = self.bm.block_size
+        return sum(1 for r in self.running
+                   if self._decoding(self.reqs[r]) and self.bm.seq_lens[r] % bs == 0)
+
+    def step(self):
+        bs = self.bm.block_size
+        info = dict(step=self.steps, num_admitted=0, num_preempted=0, num_finished=0)
+        keep = []
+        for r in self.running:
+            if self.reqs[r].state == FINISHED:
+                self.bm.free(r)
+                info["num_finished"] += 1
+            else:
+                keep.append(r)
+        self.running = keep
+        need = self._need()
+        while need > self.bm._available() and self.running:
+            v = self.running.pop()
+            q = self.reqs[v]
+            self.bm.free(v)
+            q.to_prefill = q.prompt_len + q.generated
+            q.prefilled = 0
+            q.state = WAITING
+            q.preemptions += 1
+            self.waiting.appendleft(v)
+            info["num_preempted"] += 1
+            need = self._need()
+        while len(self.running) < self.max_num_seqs and self.waiting:
+            r = self.waiting[0]
+            q = self.reqs[r]
+            if self.bm._available() - need - self.watermark < blocks_needed(q.to_prefill, bs):
+                break
+            self.waiting.popleft()
+            assert self.bm.allocate(r, 0) == OK
+            q.state = RUNNING
+            q.prefilled = 0
+            self.running.append(r)
+            info["num_admitted"] += 1
+        self.last_prefill, self.last_decode = [], []
+        dec_slots, pre_slots = [], []
+        for r in self.running:
+            if not self._decoding(self.reqs[r]):
+                continue
+            st, slot = self.bm.append_token(r)
+            assert st == OK
+            dec_slots.append(slot)
+            self.last_decode.append((r, self.bm.seq_lens[r]))
+        budget = self.max_num_tokens
+        for r in self.running:
+            q = self.reqs[r]
+            if q.state != RUNNING or q.prefilled >= q.to_prefill:
+                continue
+            remaining = q.to_prefill - q.prefilled
+            chunk = min(remaining, budget) if self.chunked else (remaining if remaining <= budget else 0)
+            if chunk <= 0:
+                continue
+            st, slots = self.bm.append_tokens(r, chunk)
+            if st == OOM:
+                continue
+            pre_slots += slots
+            self.last_prefill.append((r, q.prefilled, chunk))
+            budget -= chunk
+        info.update(num_prefill=len(self.last_prefill), num_decode=len(self.last_decode),
+                    num_tokens=len(pre_slots) + len(dec_slots),
+                    prefill=list(self.last_prefill), decode=list(self.last_decode),
+                    slot_mapping=pre_slots + dec_slots)
+        return info
+
+    def complete(self):
+        now = self.steps
+
+        def emit(q):
+            q.generated += 1
+            if q.first_token_step < 0:
+                q.first_token_step = now
+            if q.generated >= q.max_new:
+                q.state = FINISHED
+                q.finish_step = now
+
+        for r, ctx, chunk in self.last_prefill:
+            q = self.reqs[r]
+            q.prefilled += chunk
+            if q.prefilled == q.to_prefill:
+                emit(q)
+        for r, _ in self.last_decode:
+            emit(self.reqs[r])
+        self.steps += 1

@@ -22,7 +22,7 @@ from ._lib import (PA_DEVCHK_BLOCK_ID, PA_DEVCHK_QUERY_RANGE, PA_DEVCHK_SEQ_LEN,
                    CacheStats, PagedKVError, check, last_error, lib)
 
 __all__ = [
-    "BlockAllocator", "reshape_and_cache", "paged_attention_decode", "paged_attention_prefill_chunk",
+    "BlockAllocator", "Scheduler", "reshape_and_cache", "paged_attention_decode", "paged_attention_prefill_chunk",
     "decode_workspace_bytes", "paged_attention_decode_noalloc", "swap_blocks", "swap_out", "swap_in",
     "PagedKVError", "lib", "STATUS_NAMES", "PA_OK", "PA_ERR_INVALID_ARG",
     "PA_ERR_OOM", "PA_ERR_NOT_FOUND", "PA_ERR_EXISTS", "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA",
@@ -145,6 +145,64 @@ class BlockAllocator:
         out = np.empty(n.value, dtype=np.int32)
         check(lib().pa_alloc_evictable_list(self._h, _i32p(out), n.value, byref(n)))
         return out
+
+
+# ------------------------------------------------------------------ scheduler
+class Scheduler:
+    """Continuous-batching step driver (pa_sched_*) over a BlockAllocator."""
+
+    def __init__(self, alloc: "BlockAllocator", max_num_seqs: int, max_num_tokens: int, chunked_prefill: bool = True,
+                 watermark_blocks: int = 0):
+        from ._lib import SchedConfig
+        self._alloc = alloc                       # the C scheduler borrows it
+        self.max_num_seqs, self.max_num_tokens = int(max_num_seqs), int(max_num_tokens)
+        cfg = SchedConfig(self.max_num_seqs, self.max_num_tokens, int(bool(chunked_prefill)), int(watermark_blocks))
+        self._h = c_void_p()
+        check(lib().pa_sched_create(alloc._h, byref(cfg), byref(self._h)))
+
+    def close(self):
+        if self._h:
+            lib().pa_sched_destroy(self._h)
+            self._h = c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def add_request(self, req: int, prompt_len: int, max_new_tokens: int) -> int:
+        return lib().pa_sched_add_request(self._h, req, prompt_len, max_new_tokens)
+
+    def step(self) -> dict:
+        """Schedule one step; returns info plus the prefill/decode entries and the slot mapping."""
+        from ._lib import StepInfo
+        n, t = self.max_num_seqs, self.max_num_tokens + self.max_num_seqs
+        pr, pc, pl = np.empty(n, np.int64), np.empty(n, np.int32), np.empty(n, np.int32)
+        dr, dl, sm = np.empty(n, np.int64), np.empty(n, np.int32), np.empty(t, np.int64)
+        info = StepInfo()
+        check(lib().pa_sched_step(self._h, byref(info), _i64p(pr), _i32p(pc), _i32p(pl), _i64p(dr), _i32p(dl),
+                                  _i64p(sm)))
+        d = info.as_dict()
+        P, D, T = info.num_prefill, info.num_decode, info.num_tokens
+        d.update(prefill_reqs=pr[:P].copy(), prefill_ctx=pc[:P].copy(), prefill_len=pl[:P].copy(),
+                 decode_reqs=dr[:D].copy(), decode_seq_lens=dl[:D].copy(), slot_mapping=sm[:T].copy())
+        return d
+
+    def complete(self) -> None:
+        check(lib().pa_sched_complete(self._h))
+
+    def request_info(self, req: int):
+        from ._lib import RequestInfo
+        r = RequestInfo()
+        st = lib().pa_sched_request_info(self._h, req, byref(r))
+        return st, (r.as_dict() if st == PA_OK else None)
+
+    def stats(self) -> dict:
+        from ._lib import SchedStats
+        s = SchedStats()
+        check(lib().pa_sched_stats(self._h, byref(s)))
+        return s.as_dict()
 
 
 # ------------------------------------------------------------------ swapping

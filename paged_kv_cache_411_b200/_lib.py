@@ -60,6 +60,36 @@ class CacheStats(ctypes.Structure):
         return {k: getattr(self, k) for k, _ in self._fields_}
 
 
+class SchedConfig(ctypes.Structure):
+    _fields_ = [("max_num_seqs", c_int32), ("max_num_tokens", c_int32), ("chunked_prefill", c_int32),
+                ("watermark_blocks", c_int32)]
+
+
+class StepInfo(ctypes.Structure):
+    _fields_ = [("step", c_int64), ("num_prefill", c_int32), ("num_decode", c_int32), ("num_tokens", c_int32),
+                ("num_admitted", c_int32), ("num_preempted", c_int32), ("num_finished", c_int32)]
+
+    def as_dict(self):
+        return {k: getattr(self, k) for k, _ in self._fields_}
+
+
+class RequestInfo(ctypes.Structure):
+    _fields_ = [("state", c_int32), ("prompt_len", c_int32), ("max_new_tokens", c_int32), ("prefilled", c_int32),
+                ("to_prefill", c_int32), ("generated", c_int32), ("preemptions", c_int32), ("pad_", c_int32),
+                ("first_token_step", c_int64), ("finish_step", c_int64)]
+
+    def as_dict(self):
+        return {k: getattr(self, k) for k, _ in self._fields_ if k != "pad_"}
+
+
+class SchedStats(ctypes.Structure):
+    _fields_ = [(k, c_int64) for k in ("steps", "waiting", "running", "finished", "preemptions",
+                                        "prefill_tokens", "decode_tokens")]
+
+    def as_dict(self):
+        return {k: getattr(self, k) for k, _ in self._fields_}
+
+
 _P = c_void_p
 _I32P = POINTER(c_int32)
 _I64P = POINTER(c_int64)
@@ -90,6 +120,13 @@ SIGNATURES = {
     "pa_swap_blocks": (c_int32, [_P, _P, _P, _P, _I64P, c_int32, c_int64, c_int32, c_int32, _P]),
     "pa_alloc_swap_out": (c_int32, [_P, _P, c_int64, _P, _P, _P, _P, c_int64, _P]),
     "pa_alloc_swap_in": (c_int32, [_P, _P, c_int64, _P, _P, _P, _P, c_int64, _P]),
+    "pa_sched_create": (c_int32, [_P, POINTER(SchedConfig), POINTER(c_void_p)]),
+    "pa_sched_destroy": (None, [_P]),
+    "pa_sched_add_request": (c_int32, [_P, c_int64, c_int32, c_int32]),
+    "pa_sched_step": (c_int32, [_P, POINTER(StepInfo), _I64P, _I32P, _I32P, _I64P, _I32P, _I64P]),
+    "pa_sched_complete": (c_int32, [_P]),
+    "pa_sched_request_info": (c_int32, [_P, c_int64, POINTER(RequestInfo)]),
+    "pa_sched_stats": (c_int32, [_P, POINTER(SchedStats)]),
     "pa_reshape_and_cache": (c_int32, [_P, _P, _P, _P, _P, c_int32, c_int32, c_int32, c_int32, c_int32, _P, _P]),
     "pa_decode_workspace_bytes": (c_size_t, [c_int32, c_int32, c_int32, c_int32, c_int32]),
     "pa_paged_attention_decode": (c_int32, [_P, _P, _P, _P, _P, _P, c_int32, c_int32, c_int32, c_int32, c_int32,

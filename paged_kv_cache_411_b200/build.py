@@ -28,6 +28,7 @@ SOURCES = [
     "capi.cpp",
     "runtime.cpp",
     "swap.cpp",
+    "scheduler.cpp",
     "reshape_and_cache.cu",
     "decode.cu",
     "decode_noalloc.cu",

@@ -1,0 +1,115 @@
+"""Continuous-batching step driver: the C++ scheduler against the oracle scheduler, plan for
+plan, on seeded arrival traces (no GPU), plus hand-checked behaviours of the page's loop."""
+import numpy as np
+import pytest
+from hypothesis import given, settings
+from hypothesis import strategies as st
+
+import paged_kv_cache_411_b200 as pk
+from oracle import block_manager as obm
+from oracle import scheduler as osch
+from oracle.prefix_cache import PrefixCachingBlockManager
+
+
+def _pair(N, bs, **cfg):
+    ca = pk.BlockAllocator(N, bs)
+    cs = pk.Scheduler(ca, **cfg)
+    om = PrefixCachingBlockManager(N, bs)
+    os_ = osch.Scheduler(om, cfg["max_num_seqs"], cfg["max_num_tokens"], cfg.get("chunked_prefill", True),
+                         cfg.get("watermark_blocks", 0))
+    return ca, cs, om, os_
+
+
+def _run(trace, N, bs, steps, **cfg):
+    """trace: [(arrival_step, prompt_len, max_new)], request ids = index."""
+    ca, cs, om, os_ = _pair(N, bs, **cfg)
+    pending = sorted(range(len(trace)), key=lambda i: trace[i][0])
+    k = 0
+    log = []
+    for step in range(steps):
+        while k < len(pending) and trace[pending[k]][0] <= step:
+            i = pending[k]
+            assert cs.add_request(i, trace[i][1], trace[i][2]) == pk.PA_OK
+            os_.add_request(i, trace[i][1], trace[i][2])
+            k += 1
+        a = cs.step()
+        b = os_.step()
+        for key in ("num_prefill", "num_decode", "num_tokens", "num_admitted", "num_preempted", "num_finished"):
+            assert a[key] == b[key], (step, key, a[key], b[key])
+        assert [(int(r), int(c), int(n)) for r, c, n in zip(a["prefill_reqs"], a["prefill_ctx"], a["prefill_len"])] \
+            == b["prefill"]
+        assert [(int(r), int(n)) for r, n in zip(a["decode_reqs"], a["decode_seq_lens"])] == b["decode"]
+        assert a["slot_mapping"].tolist() == b["slot_mapping"]
+        cs.complete()
+        os_.complete()
+        log.append(a)
+    assert ca.free_list().tolist() == om.free_blocks
+    for i in range(len(trace)):
+        st_, info = cs.request_info(i)
+        if st_ == pk.PA_OK:
+            q = os_.reqs[i]
+            assert (info["state"], info["generated"], info["prefilled"], info["to_prefill"], info["preemptions"],
+                    info["first_token_step"], info["finish_step"]) == \
+                (q.state, q.generated, q.prefilled, q.to_prefill, q.preemptions, q.first_token_step, q.finish_step)
+    return cs, os_, log
+
+
+trace_st = st.lists(st.tuples(st.integers(0, 12), st.integers(1, 90), st.integers(1, 12)), min_size=1, max_size=14)
+
+
+@settings(max_examples=200, deadline=None)
+@given(trace_st, st.integers(4, 40), st.sampled_from([1, 4, 16]), st.integers(1, 6), st.integers(1, 64),
+       st.booleans(), st.integers(0, 2))
+def test_cpp_scheduler_matches_oracle(trace, N, bs, max_seqs, max_tokens, chunked, watermark):
+    _run(trace, N, bs, 40, max_num_seqs=max_seqs, max_num_tokens=max_tokens, chunked_prefill=chunked,
+         watermark_blocks=watermark)
+
+
+def test_seeded_trace_serves_everything():
+    """A seeded trace (lognormal prompt/output lengths, Poisson arrivals) on a pool large enough:
+    every request finishes, each emits exactly max_new tokens, and prefill/decode mix in steps."""
+    rng = np.random.default_rng(4)
+    n = 40
+    arrivals = np.cumsum(rng.poisson(0.7, n))
+    prompts = np.clip(rng.lognormal(4.0, 0.8, n).astype(int), 1, 600)
+    outs = np.clip(rng.lognormal(3.0, 0.7, n).astype(int), 1, 120)
+    trace = list(zip(arrivals.tolist(), prompts.tolist(), outs.tolist()))
+    cs, os_, log = _run(trace, 400, 16, 400, max_num_seqs=16, max_num_tokens=256)
+    stats = cs.stats()
+    assert stats["finished"] == n and stats["decode_tokens"] + n == int(outs.sum())
+    assert any(s["num_prefill"] and s["num_decode"] for s in log)      # mixed steps ([CB-PA] §2.2)
+    assert all(s["num_tokens"] - s["num_decode"] <= 256 for s in log)   # prefill budget
+
+
+def test_preemption_recomputes_newest_first():
+    """A pool too small for two long generations: the newer request is preempted, goes back to the
+    front of the waiting queue, and later recomputes its prompt plus what it had generated."""
+    cs, os_, log = _run([(0, 16, 40), (0, 16, 40)], 10, 8, 200, max_num_seqs=2, max_num_tokens=64)
+    assert sum(s["num_preempted"] for s in log) >= 1
+    q = os_.reqs[1]
+    assert q.preemptions >= 1 and q.state == osch.FINISHED and os_.reqs[0].state == osch.FINISHED
+    assert q.to_prefill > 16                                              # prompt + generated tokens
+
+
+def test_whole_prompt_mode_skips_prompts_that_do_not_fit():
+    cs, os_, log = _run([(0, 100, 2), (0, 10, 2)], 64, 16, 10, max_num_seqs=4, max_num_tokens=64,
+                        chunked_prefill=False)
+    first = log[0]
+    assert first["prefill_reqs"].tolist() == [1]      # the 100-token prompt never fits a 64-token budget
+    assert os_.reqs[0].prefilled == 0
+
+
+def test_scheduler_errors():
+    a = pk.BlockAllocator(8, 16)
+    s = pk.Scheduler(a, max_num_seqs=2, max_num_tokens=32)
+    assert s.add_request(1, 0, 5) == pk.PA_ERR_INVALID_ARG
+    assert s.add_request(1, 5, 5) == pk.PA_OK
+    assert s.add_request(1, 5, 5) == pk.PA_ERR_EXISTS
+    s.step()
+    with pytest.raises(pk.PagedKVError):
+        s.step()                                        # previous step not completed
+    s.complete()
+    with pytest.raises(pk.PagedKVError):
+        s.complete()
+    with pytest.raises(pk.PagedKVError):
+        pk.Scheduler(a, max_num_seqs=0, max_num_tokens=32)

@@ -1,0 +1,97 @@
+"""The continuous-batching step driver running the kernels (GPU).
+
+The C++ scheduler plans every step of a seeded arrival trace (mixed prefill
+chunks and decodes, preemption by recomputation under a small pool); each
+step writes its rows with reshape_and_cache and runs the prefill and decode
+kernels on the planned tables.  Every output row is checked against the
+float64 oracle's attention over the request's logical K/V (a recomputed
+position gets the same K/V, as recomputation would give)."""
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_411_b200 as pk
+from oracle import attention as oatt
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-3
+
+
+def test_scheduler_drives_kernels(cuda_ready):
+    H, D, bs, N = 4, 128, 16, 14            # a pool that forces preemptions
+    scale = 1 / np.sqrt(D)
+    rng = np.random.default_rng(30)
+    n = 10
+    prompts = rng.integers(5, 150, n)
+    outs = rng.integers(2, 24, n)
+    arrivals = np.sort(rng.integers(0, 6, n))
+    maxlen = int((prompts + outs).max()) + 1
+    K = {r: rng.standard_normal((maxlen, H, D)).astype(np.float16) for r in range(n)}
+    V = {r: rng.standard_normal((maxlen, H, D)).astype(np.float16) for r in range(n)}
+    alloc = pk.BlockAllocator(N, bs)
+    sched = pk.Scheduler(alloc, max_num_seqs=6, max_num_tokens=64)
+    kc = torch.full((N, bs, H, D), float("nan"), dtype=torch.float16, device="cuda")
+    vc = torch.full_like(kc, float("nan"))
+    mb = -(-maxlen // bs)
+    ws = torch.empty(pk.decode_workspace_bytes(6, H, D, mb, bs), dtype=torch.uint8, device="cuda")
+    added, checked_rows, preempted, mixed = 0, 0, 0, 0
+    for step in range(400):
+        while added < n and arrivals[added] <= step:
+            assert sched.add_request(added, int(prompts[added]), int(outs[added])) == pk.PA_OK
+            added += 1
+        plan = sched.step()
+        preempted += plan["num_preempted"]
+        if plan["num_tokens"] == 0:
+            sched.complete()
+            if sched.stats()["finished"] == n:
+                break
+            continue
+        mixed += bool(plan["num_prefill"] and plan["num_decode"])
+        rows = []                                           # (request, position) of each slot-mapping row
+        for r, c, L in zip(plan["prefill_reqs"], plan["prefill_ctx"], plan["prefill_len"]):
+            rows += [(int(r), p) for p in range(int(c), int(c) + int(L))]
+        for r, sl in zip(plan["decode_reqs"], plan["decode_seq_lens"]):
+            rows.append((int(r), int(sl) - 1))
+        k_rows = np.stack([K[r][p] for r, p in rows])
+        v_rows = np.stack([V[r][p] for r, p in rows])
+        pk.reshape_and_cache(torch.from_numpy(k_rows).cuda(), torch.from_numpy(v_rows).cuda(), kc, vc,
+                             torch.from_numpy(plan["slot_mapping"]).cuda())
+        P, S = plan["num_prefill"], plan["num_decode"]
+        if P:
+            T = int(plan["prefill_len"].sum())
+            qp = rng.standard_normal((T, H, D)).astype(np.float16)
+            st, tables, _ = alloc.pack(plan["prefill_reqs"], mb)
+            assert st == pk.PA_OK
+            q_start = np.concatenate([[0], np.cumsum(plan["prefill_len"])]).astype(np.int32)
+            out = torch.empty(T, H, D, dtype=torch.float16, device="cuda")
+            pk.paged_attention_prefill_chunk(out, torch.from_numpy(qp).cuda(), kc, vc, torch.from_numpy(tables).cuda(),
+                                             torch.from_numpy(q_start).cuda(),
+                                             torch.from_numpy(plan["prefill_ctx"]).cuda(), scale)
+            got = out.float().cpu().numpy()
+            for i, (r, c, L) in enumerate(zip(plan["prefill_reqs"], plan["prefill_ctx"], plan["prefill_len"])):
+                r, c, L = int(r), int(c), int(L)
+                allowed = np.arange(c + L)[None, :] <= (c + np.arange(L))[:, None]
+                ref = oatt.softmax_attention(qp[q_start[i]:q_start[i + 1]], K[r][:c + L], V[r][:c + L], scale, allowed)
+                assert np.abs(got[q_start[i]:q_start[i + 1]] - ref).max() <= TOL, (step, r)
+                checked_rows += L
+        if S:
+            qd = rng.standard_normal((S, H, D)).astype(np.float16)
+            st, tables, lens = alloc.pack(plan["decode_reqs"], mb)
+            assert st == pk.PA_OK and lens.tolist() == plan["decode_seq_lens"].tolist()
+            out = torch.empty(S, H, D, dtype=torch.float16, device="cuda")
+            pk.paged_attention_decode(out, torch.from_numpy(qd).cuda(), kc, vc, torch.from_numpy(tables).cuda(),
+                                      torch.from_numpy(lens).cuda(), scale, ws)
+            got = out.float().cpu().numpy()
+            for i, (r, sl) in enumerate(zip(plan["decode_reqs"], plan["decode_seq_lens"])):
+                r, sl = int(r), int(sl)
+                ref = oatt.softmax_attention(qd[i][None], K[r][:sl], V[r][:sl], scale)[0]
+                assert np.abs(got[i] - ref).max() <= TOL, (step, r)
+                checked_rows += 1
+        sched.complete()
+        if sched.stats()["finished"] == n:
+            break
+    stats = sched.stats()
+    assert stats["finished"] == n and preempted > 0 and mixed > 0 and checked_rows > 500
+    for r in range(n):
+        st, info = sched.request_info(r)
+        assert info["generated"] == outs[r]
