@@ -52,7 +52,9 @@ namespace pagedkv {
 namespace {
 
 constexpr int kConsumerWarps = 16;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kProducer = kConsumerWarps;          // warp index of the TMA producer
+constexpr int kEpilogue = kConsumerWarps + 1;      // warp index of the epilogue
+constexpr int kThreads = (kConsumerWarps + 2) * 32;
 constexpr int kStageTok = 16;
 constexpr int kMinSplit = 64;
 constexpr int kSmemBudget = 192 * 1024;          // K + V stage ring
@@ -119,16 +121,15 @@ struct Cfg {
     static constexpr int kStagesRaw = kSmemBudget / (2 * kTileBytes);
     static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
     static constexpr int kQBytes = HG * D * 2;
-    static constexpr int kMergeSlots = HG * (kWPH - 1);         // warps that hand their state over
-    static constexpr int kMergeStride = D + 4;                   // floats per slot: acc[D], m, l, pad
-    static constexpr int kMergeFloats = kMergeSlots * kMergeStride;
+    static constexpr int kHandStride = D + 4;                    // floats per warp: acc[D], m, l, pad
+    static constexpr int kHandFloats = kConsumerWarps * kHandStride;   // one hand-off slot
     static constexpr size_t kOffK = 0;
     static constexpr size_t kOffV = kOffK + size_t(kStages) * kTileBytes;
     static constexpr size_t kOffQ = kOffV + size_t(kStages) * kTileBytes;
-    static constexpr size_t kOffMerge = kOffQ + size_t(kStages) * kQBytes;
-    static constexpr size_t kOffInfo = kOffMerge + size_t(2) * kMergeFloats * 4;
-    static constexpr size_t kOffBar = (kOffInfo + size_t(kStages) * 16 + 15) & ~size_t(15);
-    static constexpr size_t kNumBars = 3 * kStages + 2;
+    static constexpr size_t kOffHand = kOffQ + size_t(kStages) * kQBytes;
+    static constexpr size_t kOffInfo = kOffHand + size_t(2) * kHandFloats * 4;    // stage infos, then 2 hand-off infos
+    static constexpr size_t kOffBar = (kOffInfo + size_t(kStages + 2) * 16 + 15) & ~size_t(15);
+    static constexpr size_t kNumBars = 3 * kStages + 4;
     static constexpr size_t kOffAbort = kOffBar + kNumBars * 8;
     static constexpr size_t kSmemBytes = kOffAbort + 16 + 1024;   // + alignment slack
     static_assert(kWPH >= 1 && kTPW >= kTPL && kTPW % kTPL == 0, "bad warp split");
@@ -332,12 +333,14 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     uint8_t* tile_k = smem + C::kOffK;
     uint8_t* tile_v = smem + C::kOffV;
     uint8_t* qbuf = smem + C::kOffQ;
-    float* merge = reinterpret_cast<float*>(smem + C::kOffMerge);
+    float* hand = reinterpret_cast<float*>(smem + C::kOffHand);
     int4* info = reinterpret_cast<int4*>(smem + C::kOffInfo);
     uint64_t* full_k = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* full_v = full_k + C::kStages;
     uint64_t* empty = full_v + C::kStages;
-    uint64_t* merge_bar = empty + C::kStages;
+    int4* hand_info = info + C::kStages;
+    uint64_t* hand_full = empty + C::kStages;     // [2] every consumer warp has handed its state over
+    uint64_t* hand_empty = hand_full + 2;         // [2] the epilogue has read the slot
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffAbort);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -347,8 +350,10 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             mbar_init(&full_v[s], 1);
             mbar_init(&empty[s], kConsumerWarps);
         }
-        mbar_init(&merge_bar[0], kConsumerWarps);
-        mbar_init(&merge_bar[1], kConsumerWarps);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&hand_full[i], kConsumerWarps);
+            mbar_init(&hand_empty[i], 1);
+        }
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -357,7 +362,7 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 
     const int n_items = p.hdr[1];
 
-    if (warp == kConsumerWarps) {
+    if (warp == kProducer) {
         // ================================================= producer warp
         if (lane == 0) {
             tma_prefetch_desc(&tm_k);
@@ -450,6 +455,82 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         return;
     }
 
+    if (warp == kEpilogue) {
+        // ================================================= epilogue warp
+        // Per finished item: merge the warps of each head, then write the output (single-partition
+        // sequences) or the fp32 partial, publish it and take the (sequence, head) ticket; the
+        // partial that takes the last ticket merges all partitions.  Off the streaming path.
+        constexpr int VEC = D / 32;
+        uint32_t uses = 0;
+        while (true) {
+            const int hs = uses & 1;
+            if (!mbar_wait(&hand_full[hs], (uses >> 1) & 1)) {
+                flag_error(p.err_flag, kDevchkTimeout);
+                *abort_flag = 1;
+                break;
+            }
+            const int4 inf = hand_info[hs];
+            if (inf.w & kTerminate) break;
+            const int seq = inf.x, part = inf.y & 0xffff, nsp = inf.y >> 16, hg = inf.z;
+            const float* hb = hand + hs * C::kHandFloats;
+            float accs[HG][VEC];
+            float Ms[HG], Ls[HG];
+#pragma unroll
+            for (int hh = 0; hh < HG; ++hh) {
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < C::kWPH; ++w) M = fmaxf(M, hb[(hh * C::kWPH + w) * C::kHandStride + D]);
+                const float Mu = M == -INFINITY ? 0.f : M;
+                float L = 0.f;
+#pragma unroll
+                for (int k = 0; k < VEC; ++k) accs[hh][k] = 0.f;
+#pragma unroll
+                for (int w = 0; w < C::kWPH; ++w) {
+                    const float* ws_ = hb + (hh * C::kWPH + w) * C::kHandStride;
+                    const float wt = exp2f(ws_[D] - Mu);
+                    L = fmaf(ws_[D + 1], wt, L);
+#pragma unroll
+                    for (int k = 0; k < VEC; ++k) accs[hh][k] = fmaf(ws_[lane * VEC + k], wt, accs[hh][k]);
+                }
+                Ms[hh] = M;
+                Ls[hh] = L;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&hand_empty[hs]);
+            ++uses;
+            if (nsp == 1) {
+#pragma unroll
+                for (int hh = 0; hh < HG; ++hh) {
+                    const float r = 1.f / Ls[hh];
+                    __half* o = p.out + (static_cast<int64_t>(seq) * p.H + hg * HG + hh) * D + lane * VEC;
+#pragma unroll
+                    for (int k = 0; k < VEC; k += 2) *reinterpret_cast<uint32_t*>(o + k) = f2_to_h2(accs[hh][k] * r, accs[hh][k + 1] * r);
+                }
+                continue;
+            }
+#pragma unroll
+            for (int hh = 0; hh < HG; ++hh) {
+                const int64_t pi = (static_cast<int64_t>(seq) * p.max_splits + part) * p.H + hg * HG + hh;
+                float* dst = p.part_acc + pi * D + lane * VEC;
+#pragma unroll
+                for (int k = 0; k < VEC; ++k) dst[k] = accs[hh][k];
+                if (lane == 0) p.part_ml[pi] = make_float2(Ms[hh], Ls[hh]);
+            }
+            // publish the partials, then take one ticket per head (lanes 0..HG-1)
+            __threadfence();
+            __syncwarp();
+            int ticket = -1;
+            if (lane < HG) ticket = atomicAdd(&p.tickets[static_cast<int64_t>(seq) * p.H + hg * HG + lane], 1);
+            const unsigned last = __ballot_sync(0xffffffffu, lane < HG && ticket == nsp - 1);
+            if (last) {
+                __threadfence();
+                for (int hh = 0; hh < HG; ++hh)
+                    if ((last >> hh) & 1u) combine_head<D>(p, seq, hg * HG + hh, nsp, lane);
+            }
+        }
+        return;
+    }
+
     // ===================================================== consumer warps
     const int hh = warp / C::kWPH;        // head within the group
     const int ww = warp % C::kWPH;        // slice of the stage's tokens
@@ -461,12 +542,21 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     float qf[8];
     float acc[8];
     float m_run = -INFINITY, l_lane = 0.f;
-    uint32_t stage = 0, phase = 0, merge_uses = 0;
+    uint32_t stage = 0, phase = 0, hand_uses = 0;
     while (true) {
         if (!mbar_wait(&full_k[stage], phase)) { flag_error(p.err_flag, kDevchkTimeout); *abort_flag = 1; break; }
         const int4 inf = info[stage];
         const int flags = inf.w;
-        if (flags & kTerminate) break;
+        if (flags & kTerminate) {
+            // tell the epilogue warp there is nothing more to merge
+            const int hs = hand_uses & 1;
+            if (mbar_wait(&hand_empty[hs], ((hand_uses >> 1) & 1) ^ 1)) {
+                if (warp == 0 && lane == 0) hand_info[hs] = make_int4(0, 0, 0, kTerminate);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&hand_full[hs]);
+            }
+            break;
+        }
         const int ntok = flags & 0xff;
         const uint8_t* tk = tile_k + size_t(stage) * C::kTileBytes;
         const uint8_t* tv = tile_v + size_t(stage) * C::kTileBytes;
@@ -516,7 +606,7 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         if (lane == 0) mbar_arrive(&empty[stage]);
 
         if (flags & kLast) {
-            // ---- finish the item: fold the token rows, then the warps of this head.
+            // ---- finish the item: fold the token rows and hand (m, l, acc) to the epilogue warp.
             float a8[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
@@ -529,70 +619,21 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 #pragma unroll
             for (int off = 16; off >= 1; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
             l *= 1.0f / C::kRep;
-            const int par = merge_uses & 1;
-            float* mb = merge + par * C::kMergeFloats;
-            if (C::kWPH > 1 && ww > 0) {
-                float* slot = mb + (hh * (C::kWPH - 1) + (ww - 1)) * C::kMergeStride;
-                if (tq == 0) {
-                    *reinterpret_cast<float4*>(slot + sub * 8) = make_float4(a8[0], a8[1], a8[2], a8[3]);
-                    *reinterpret_cast<float4*>(slot + sub * 8 + 4) = make_float4(a8[4], a8[5], a8[6], a8[7]);
-                }
-                if (lane == 0) { slot[D] = m_run; slot[D + 1] = l; }
+            const int hs = hand_uses & 1;
+            if (!mbar_wait(&hand_empty[hs], ((hand_uses >> 1) & 1) ^ 1)) { flag_error(p.err_flag, kDevchkTimeout); *abort_flag = 1; break; }
+            float* slot = hand + hs * C::kHandFloats + warp * C::kHandStride;
+            if (tq == 0) {
+                *reinterpret_cast<float4*>(slot + sub * 8) = make_float4(a8[0], a8[1], a8[2], a8[3]);
+                *reinterpret_cast<float4*>(slot + sub * 8 + 4) = make_float4(a8[4], a8[5], a8[6], a8[7]);
+            }
+            if (lane == 0) {
+                slot[D] = m_run;
+                slot[D + 1] = l;
+                if (warp == 0) hand_info[hs] = inf;
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&merge_bar[par]);
-            if (!mbar_wait(&merge_bar[par], (merge_uses >> 1) & 1)) { flag_error(p.err_flag, kDevchkTimeout); *abort_flag = 1; break; }
-            ++merge_uses;
-            if (ww == 0) {
-                float M = m_run;
-                for (int j = 1; j < C::kWPH; ++j) M = fmaxf(M, mb[(hh * (C::kWPH - 1) + (j - 1)) * C::kMergeStride + D]);
-                const float Mu = M == -INFINITY ? 0.f : M;
-                float w0 = exp2f(m_run - Mu);
-                float L = l * w0;
-#pragma unroll
-                for (int k = 0; k < 8; ++k) a8[k] *= w0;
-                for (int j = 1; j < C::kWPH; ++j) {
-                    const float* slot = mb + (hh * (C::kWPH - 1) + (j - 1)) * C::kMergeStride;
-                    const float wj = exp2f(slot[D] - Mu);
-                    L = fmaf(slot[D + 1], wj, L);
-                    const float4 x = *reinterpret_cast<const float4*>(slot + sub * 8);
-                    const float4 y = *reinterpret_cast<const float4*>(slot + sub * 8 + 4);
-                    a8[0] = fmaf(x.x, wj, a8[0]); a8[1] = fmaf(x.y, wj, a8[1]);
-                    a8[2] = fmaf(x.z, wj, a8[2]); a8[3] = fmaf(x.w, wj, a8[3]);
-                    a8[4] = fmaf(y.x, wj, a8[4]); a8[5] = fmaf(y.y, wj, a8[5]);
-                    a8[6] = fmaf(y.z, wj, a8[6]); a8[7] = fmaf(y.w, wj, a8[7]);
-                }
-                const int seq = inf.x, part = inf.y & 0xffff, nsp = inf.y >> 16, head = inf.z * HG + hh;
-                if (flags & kSingle) {
-                    if (tq == 0) {
-                        const float r = 1.f / L;
-                        uint4 o;
-                        o.x = f2_to_h2(a8[0] * r, a8[1] * r);
-                        o.y = f2_to_h2(a8[2] * r, a8[3] * r);
-                        o.z = f2_to_h2(a8[4] * r, a8[5] * r);
-                        o.w = f2_to_h2(a8[6] * r, a8[7] * r);
-                        *reinterpret_cast<uint4*>(p.out + (static_cast<int64_t>(seq) * p.H + head) * D + sub * 8) = o;
-                    }
-                } else {
-                    const int64_t pi = (static_cast<int64_t>(seq) * p.max_splits + part) * p.H + head;
-                    if (tq == 0) {
-                        float* dst = p.part_acc + pi * D + sub * 8;
-                        *reinterpret_cast<float4*>(dst) = make_float4(a8[0], a8[1], a8[2], a8[3]);
-                        *reinterpret_cast<float4*>(dst + 4) = make_float4(a8[4], a8[5], a8[6], a8[7]);
-                    }
-                    if (lane == 0) p.part_ml[pi] = make_float2(M, L);
-                    // Publish the partial, then take a ticket; the last partition merges them all.
-                    __threadfence();
-                    __syncwarp();
-                    int ticket = 0;
-                    if (lane == 0) ticket = atomicAdd(&p.tickets[static_cast<int64_t>(seq) * p.H + head], 1);
-                    ticket = __shfl_sync(0xffffffffu, ticket, 0);
-                    if (ticket == nsp - 1) {
-                        __threadfence();
-                        combine_head<D>(p, seq, head, nsp, lane);
-                    }
-                }
-            }
+            if (lane == 0) mbar_arrive(&hand_full[hs]);
+            ++hand_uses;
         }
         if (*abort_flag) break;
         if (++stage == C::kStages) { stage = 0; phase ^= 1; }
