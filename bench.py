@@ -366,13 +366,13 @@ def run_ours(args):
             "pct_of_nominal_8tbs": round(100 * value / world / 8000.0, 2),
             "decode_tokens_per_s": round(S * world / (ms_per_step / 1e3), 1),
             "decode_tokens_per_s_32_layers": round(S * world / (32 * ms_per_step / 1e3), 1),
-            "roofline": {"kernel": "paged_attention_decode (plan + streaming kernel with in-kernel combine)", "bound": "hbm",
+            "roofline": {"kernel": "paged_attention_decode (plan + streaming kernel + combine)", "bound": "hbm",
                          "achieved": round(dec_gbs, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": round(dec_gbs / peak, 4), "traffic": None,
                          "algorithmic_bytes_per_launch": dec_b, "avg_launch_ms": round(dec_avg_ms, 5)},
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(1e3 * e2e_max / args.steps, 4)},
-            "gpu_launches": args.steps * (3 + (1 if pout is not None else 0)),
+            "gpu_launches": args.steps * (4 + (1 if pout is not None else 0)),
             "kv_pool": pool_stats(ds),
             "clocks": clk.summary(),
         }

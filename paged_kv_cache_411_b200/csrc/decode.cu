@@ -30,14 +30,15 @@
 //     transposing warp-shuffle reduction, and P.V accumulates in registers.
 //     The warps sharing a head merge their (max, sum, acc) through shared
 //     memory at the end of the item; single-partition sequences are written
-//     straight to `out`, others write an fp32 partial and take a ticket for
-//     their (sequence, head): the warp that takes the last ticket merges all
-//     partitions with the exact log-sum-exp rule
-//     m* = max m_i, l* = sum l_i 2^(m_i - m*), o* = sum acc_i 2^(m_i - m*) / l*
-//     and writes the output, so no separate combine launch is needed.
-//  The streaming kernel is launched as a programmatic dependent of the plan
-//  kernel: its CTAs become resident and set up their barriers and TMA
-//  descriptors while the plan runs, and wait for it with griddepcontrol.
+//     straight to `out`, others write an fp32 partial.  The consumer warps
+//     hand their (m, l, acc) to an epilogue warp through a double-buffered
+//     shared-memory slot, so the head merge and the global stores never hold
+//     up the stage ring.
+//  3. combine kernel (one warp per (sequence, head) with several partitions):
+//     m* = max m_i, l* = sum l_i 2^(m_i - m*), o* = sum acc_i 2^(m_i - m*) / l*.
+//  Each kernel is launched as a programmatic dependent of the one before: its
+//  CTAs become resident (barriers, TMA descriptors) while the previous kernel
+//  finishes, and wait for it with griddepcontrol before reading its output.
 //
 // The combine order is the partition order and the in-item merge order is
 // fixed, so the result does not depend on physical block placement (bitwise)
@@ -68,7 +69,7 @@ constexpr int kTerminate = 1 << 11;
 
 // Item record: x = seq, y = first token, z = tokens | (head group << 10), w = partition | (partitions << 16).
 struct WsLayout {
-    size_t hdr, n_splits, items, part_ml, part_acc, tickets, total;
+    size_t hdr, n_splits, items, part_ml, part_acc, total;
     int32_t max_splits;
 };
 
@@ -85,7 +86,6 @@ inline WsLayout ws_layout(int32_t S, int32_t H, int32_t D, int32_t max_blocks, i
     w.items = off;      off = align256(off + sizeof(int4) * pairs * H);
     w.part_ml = off;    off = align256(off + sizeof(float2) * pairs * H);
     w.part_acc = off;   off = align256(off + sizeof(float) * pairs * H * D);
-    w.tickets = off;    off = align256(off + sizeof(int32_t) * static_cast<size_t>(S) * H);
     w.total = off;
     return w;
 }
@@ -101,7 +101,6 @@ struct DecodeParams {
     int4* items;
     float2* part_ml;
     float* part_acc;
-    int32_t* tickets;                   // [S][H] partitions merged so far (zeroed by the plan)
     int32_t max_splits;
     int32_t* err_flag;
 };
@@ -281,8 +280,6 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeParams p, int32
                 p.items[off_p * hg_count + g] = make_int4(s, nfull * split, tail | (g << 10), nfull | (nsp << 16));
             ++off_p;
         }
-        if (nsp > 1)
-            for (int h = 0; h < p.H; ++h) p.tickets[static_cast<int64_t>(s) * p.H + h] = 0;
         if (nsp == 0) {                 // empty sequence: zeros
             uint4* o = reinterpret_cast<uint4*>(p.out + static_cast<int64_t>(s) * p.H * head_dim);
             for (int i = 0; i < p.H * head_dim / 8; ++i) o[i] = make_uint4(0, 0, 0, 0);
@@ -295,29 +292,39 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeParams p, int32
     }
 }
 
-// Merge the nsp fp32 partials of (seq, head) with the log-sum-exp rule and write the fp16 output.
-// Called by one warp, after every partial of the pair is visible (ticket protocol); reads bypass L1.
+// ---------------------------------------------------------------- combine ----
+// One warp per (sequence, head) of a multi-partition sequence: merge its fp32 partials with the
+// log-sum-exp rule, in partition order, and write the fp16 output.  Launched as a programmatic
+// dependent of the streaming kernel; waits for it before reading anything.
 template <int D>
-__device__ __forceinline__ void combine_head(const DecodeParams& p, int seq, int head, int nsp, int lane) {
+__global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
+    pdl_wait();
     constexpr int VEC = D / 32;
-    const int64_t base = static_cast<int64_t>(seq) * p.max_splits * p.H + head;
+    const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (gw >= p.S * p.H) return;
+    const int s = gw / p.H, h = gw % p.H;
+    const int n = p.n_splits[s];
+    if (n <= 1) return;
+    const int64_t base = static_cast<int64_t>(s) * p.max_splits * p.H + h;
     float M = -INFINITY;
-    for (int i = lane; i < nsp; i += 32) M = fmaxf(M, __ldcg(&p.part_ml[base + static_cast<int64_t>(i) * p.H]).x);
+    for (int i = lane; i < n; i += 32) M = fmaxf(M, p.part_ml[base + static_cast<int64_t>(i) * p.H].x);
     for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
     float L = 0.f, acc[VEC];
 #pragma unroll
     for (int k = 0; k < VEC; ++k) acc[k] = 0.f;
-    for (int i = 0; i < nsp; ++i) {
+#pragma unroll 4
+    for (int i = 0; i < n; ++i) {
         const int64_t pi = base + static_cast<int64_t>(i) * p.H;
-        const float2 ml = __ldcg(&p.part_ml[pi]);
+        const float2 ml = p.part_ml[pi];
         const float w = exp2f(ml.x - M);
         L = fmaf(ml.y, w, L);
         const float* a = p.part_acc + pi * D + lane * VEC;
 #pragma unroll
-        for (int k = 0; k < VEC; ++k) acc[k] = fmaf(__ldcg(a + k), w, acc[k]);
+        for (int k = 0; k < VEC; ++k) acc[k] = fmaf(a[k], w, acc[k]);
     }
     const float r = 1.f / L;
-    __half* o = p.out + (static_cast<int64_t>(seq) * p.H + head) * D + lane * VEC;
+    __half* o = p.out + static_cast<int64_t>(gw) * D + lane * VEC;
 #pragma unroll
     for (int k = 0; k < VEC; k += 2) *reinterpret_cast<uint32_t*>(o + k) = f2_to_h2(acc[k] * r, acc[k + 1] * r);
 }
@@ -359,6 +366,7 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     }
     __syncthreads();
     pdl_wait();                       // the plan (and everything before it) has completed
+    pdl_launch_dependents();          // the combine grid may be scheduled as our CTAs retire
 
     const int n_items = p.hdr[1];
 
@@ -458,8 +466,7 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     if (warp == kEpilogue) {
         // ================================================= epilogue warp
         // Per finished item: merge the warps of each head, then write the output (single-partition
-        // sequences) or the fp32 partial, publish it and take the (sequence, head) ticket; the
-        // partial that takes the last ticket merges all partitions.  Off the streaming path.
+        // sequences) or the fp32 partial that the combine kernel merges.  Off the streaming path.
         constexpr int VEC = D / 32;
         uint32_t uses = 0;
         while (true) {
@@ -515,17 +522,6 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 #pragma unroll
                 for (int k = 0; k < VEC; ++k) dst[k] = accs[hh][k];
                 if (lane == 0) p.part_ml[pi] = make_float2(Ms[hh], Ls[hh]);
-            }
-            // publish the partials, then take one ticket per head (lanes 0..HG-1)
-            __threadfence();
-            __syncwarp();
-            int ticket = -1;
-            if (lane < HG) ticket = atomicAdd(&p.tickets[static_cast<int64_t>(seq) * p.H + hg * HG + lane], 1);
-            const unsigned last = __ballot_sync(0xffffffffu, lane < HG && ticket == nsp - 1);
-            if (last) {
-                __threadfence();
-                for (int hh = 0; hh < HG; ++hh)
-                    if ((last >> hh) & 1u) combine_head<D>(p, seq, hg * HG + hh, nsp, lane);
             }
         }
         return;
@@ -701,7 +697,6 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream, const char**
     p.items = reinterpret_cast<int4*>(ws + w.items);
     p.part_ml = reinterpret_cast<float2*>(ws + w.part_ml);
     p.part_acc = reinterpret_cast<float*>(ws + w.part_acc);
-    p.tickets = reinterpret_cast<int32_t*>(ws + w.tickets);
     p.max_splits = w.max_splits;
     p.err_flag = a.err_flag;
     if (a.num_seqs == 0) return cudaSuccess;
@@ -738,6 +733,21 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream, const char**
     } else {
         if (HG == 8) e = run_main<64, 8>(tk, tv, tq, p, sms, stream);
         else e = run_main<64, 4>(tk, tv, tq, p, sms, stream);
+    }
+    if (e != cudaSuccess) return e;
+    {
+        const int warps = a.num_seqs * a.num_heads;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((warps + 7) / 8);
+        cfg.blockDim = dim3(256);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (a.head_dim == 128) e = cudaLaunchKernelEx(&cfg, decode_combine_kernel<128>, p);
+        else e = cudaLaunchKernelEx(&cfg, decode_combine_kernel<64>, p);
     }
     return e;
 }
