@@ -395,6 +395,112 @@ def run_ours(args):
     return 0
 
 
+def serve_trace(n, seed=2060):
+    """Seeded serving trace: all requests arrive at once (request rate inf); prompt and output lengths
+    lognormal with means near 223 and 198 tokens (the totals of the page's ShareGPT run, 223,417 input and
+    198,203 output tokens over 1000 prompts)."""
+    rng = np.random.default_rng(seed)
+    sigma = 1.0
+    prompts = np.clip(rng.lognormal(np.log(223) - sigma ** 2 / 2, sigma, n), 4, 2048).astype(int)
+    outs = np.clip(rng.lognormal(np.log(198) - sigma ** 2 / 2, sigma, n), 1, 1024).astype(int)
+    return prompts, outs
+
+
+def run_serve(args):
+    """Continuous batching over a seeded trace: the C++ scheduler plans every step, the step runs
+    reshape_and_cache, the chunked-prefill kernel and the decode kernel for one attention layer."""
+    import torch
+
+    import paged_kv_cache_411_b200 as pk
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    H, D, bs = 32, 128, 16
+    n = args.serve_requests
+    prompts, outs = serve_trace(n)
+    max_seqs, max_tokens = 256, 8192
+    N = args.serve_blocks
+    alloc = pk.BlockAllocator(N, bs)
+    sched = pk.Scheduler(alloc, max_num_seqs=max_seqs, max_num_tokens=max_tokens)
+    for r in range(n):
+        sched.add_request(r, int(prompts[r]), int(outs[r]))
+    kc = torch.zeros((N, bs, H, D), dtype=torch.float16, device=dev)
+    vc = torch.zeros_like(kc)
+    g = torch.Generator(device=dev).manual_seed(7)
+    rows = max_tokens + max_seqs
+    kpool = torch.randn((rows, H, D), generator=g, device=dev).half()
+    vpool = torch.randn((rows, H, D), generator=g, device=dev).half()
+    qpool = torch.randn((rows, H, D), generator=g, device=dev).half()
+    mb = -(-int((prompts + outs).max()) // bs)
+    ws = torch.empty(pk.decode_workspace_bytes(max_seqs, H, D, mb, bs), dtype=torch.uint8, device=dev)
+    out_d = torch.empty((max_seqs, H, D), dtype=torch.float16, device=dev)
+    out_p = torch.empty((max_tokens, H, D), dtype=torch.float16, device=dev)
+    scale = 1 / np.sqrt(D)
+    stream = torch.cuda.current_stream(dev)
+    ends, gpu_ms, host_s = [], [], 0.0
+    t_start = time.perf_counter()
+    while sched.stats()["finished"] < n:
+        h0 = time.perf_counter()
+        plan = sched.step()
+        P, S, T = plan["num_prefill"], plan["num_decode"], plan["num_tokens"]
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if T:
+            slots = torch.from_numpy(plan["slot_mapping"]).pin_memory().to(dev, non_blocking=True)
+            if P:
+                _, pt, _ = alloc.pack(plan["prefill_reqs"], mb)
+                q_start = np.concatenate([[0], np.cumsum(plan["prefill_len"])]).astype(np.int32)
+                pt_d = torch.from_numpy(pt).pin_memory().to(dev, non_blocking=True)
+                qs_d = torch.from_numpy(q_start).pin_memory().to(dev, non_blocking=True)
+                ctx_d = torch.from_numpy(plan["prefill_ctx"]).pin_memory().to(dev, non_blocking=True)
+            if S:
+                _, dt, dl = alloc.pack(plan["decode_reqs"], mb)
+                dt_d = torch.from_numpy(dt).pin_memory().to(dev, non_blocking=True)
+                dl_d = torch.from_numpy(dl).pin_memory().to(dev, non_blocking=True)
+            host_s += time.perf_counter() - h0
+            ev0.record(stream)
+            pk.reshape_and_cache(kpool[:T], vpool[:T], kc, vc, slots, stream=stream)
+            if P:
+                Tp = int(q_start[-1])
+                pk.paged_attention_prefill_chunk(out_p[:Tp], qpool[:Tp], kc, vc, pt_d, qs_d, ctx_d, scale,
+                                                 stream=stream)
+            if S:
+                pk.paged_attention_decode(out_d[:S], qpool[:S], kc, vc, dt_d, dl_d, scale, ws, stream=stream)
+            ev1.record(stream)
+            stream.synchronize()                     # the step's result goes back to the host
+            gpu_ms.append(ev0.elapsed_time(ev1))
+        sched.complete()
+        ends.append(time.perf_counter() - t_start)
+    wall = time.perf_counter() - t_start
+    ends = np.asarray(ends)
+    ttft, tpot = [], []
+    for r in range(n):
+        _, info = sched.request_info(r)
+        ttft.append(ends[info["first_token_step"]] * 1e3)
+        if info["generated"] > 1:
+            tpot.append((ends[info["finish_step"]] - ends[info["first_token_step"]]) * 1e3 / (info["generated"] - 1))
+    st = sched.stats()
+
+    def dist(x):
+        x = np.asarray(x)
+        return {"mean": round(float(x.mean()), 3), "median": round(float(np.median(x)), 3),
+                "p99": round(float(np.percentile(x, 99)), 3)}
+
+    line = {
+        "metric": "serve: output tokens/s of continuous batching over one attention layer", "impl": "ours",
+        "value": round(float(outs.sum()) / wall, 1), "unit": "tok/s", "higher_is_better": True,
+        "data": "synthetic", "dtype": "f16",
+        "config": {"workload": f"serve_trace_{n}req_rate_inf_lognormal223_198", "num_heads": H, "head_dim": D,
+                   "block_size": bs, "num_blocks": N, "max_num_seqs": max_seqs, "max_num_batched_tokens": max_tokens,
+                   "chunked_prefill": True, "input_tokens": int(prompts.sum()), "output_tokens": int(outs.sum())},
+        "wall_s": round(wall, 3), "req_per_s": round(n / wall, 2), "steps": st["steps"],
+        "preemptions": st["preemptions"], "prefill_tokens": st["prefill_tokens"],
+        "gpu_ms_total": round(float(np.sum(gpu_ms)), 2), "host_schedule_s": round(host_s, 3),
+        "ttft_ms": dist(ttft), "tpot_ms": dist(tpot),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -407,11 +513,17 @@ def main(argv=None):
     ap.add_argument("--oracle-tokens", type=int, default=40000,
                     help="cached tokens in the cpu_baseline leg's bounded sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--serve", action="store_true",
+                    help="continuous-batching run over a seeded trace instead of the single-step benchmark")
+    ap.add_argument("--serve-requests", type=int, default=1000)
+    ap.add_argument("--serve-blocks", type=int, default=7680)
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.serve:
+        return run_serve(args)
     return run_ours(args)
 
 
