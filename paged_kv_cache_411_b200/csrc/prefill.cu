@@ -10,12 +10,12 @@
 //
 // One CTA computes one tile of 128 query rows x one head (FlashAttention
 // order, online softmax over 128-key tiles):
-//   * warp 8 (producer) loads the Q tile once and streams K and V tiles into
-//     two-stage rings with TMA: a K/V tile of 128 keys is gathered from the
-//     paged pool with one 3-D box per physical block and 64-dim chunk ([box
+//   * warps 8 and 10 (producers) load the Q tile once and stream the K and the
+//     V tiles into two-stage rings with TMA: a tile of 128 keys is gathered from
+//     the paged pool with one 3-D box per (physical block, 64-dim chunk) ([box
 //     rows][1 head][64 dims], 128-byte swizzle), landing directly in the
-//     canonical UMMA layout; each lane issues its own block's boxes, and the
-//     next tile's block ids are read while the current tile's copies go out;
+//     canonical UMMA layout; each lane issues one box, so a tile is one TMA
+//     instruction, and the next tile's block ids are read a tile ahead;
 //   * warp 9 (one elected thread) issues tcgen05.mma: S = Q K^T (A and B
 //     K-major) into a double-buffered fp32 TMEM tile, and O_j = P_j V_j (B
 //     MN-major straight from the V tile) into a second double-buffered TMEM
@@ -41,9 +41,10 @@ namespace {
 
 constexpr int kTile = 128;
 constexpr int kSoftmaxWarps = 8;          // two warpgroups: each owns half of the S / O columns
-constexpr int kProducerWarp = 8;
+constexpr int kProducerWarp = 8;          // Q and K tiles
 constexpr int kMmaWarp = 9;
-constexpr int kThreadsP = 10 * 32;
+constexpr int kProducerVWarp = 10;        // V tiles
+constexpr int kThreadsP = 11 * 32;
 constexpr float kLog2eP = 1.4426950408889634f;
 
 struct PrefillParams {
@@ -187,23 +188,29 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         info[2] = 1;
     };
 
-    if (warp == kProducerWarp) {
-        // ======================================================= TMA producer
+    if (warp == kProducerWarp || warp == kProducerVWarp) {
+        // ======================================================= TMA producers (K warp, V warp)
+        // A 128-key tile is one box per (physical block, 64-dim chunk): lane L issues box L of the tile,
+        // so a tile goes out as one TMA instruction.  The next tile's block ids are read while the
+        // current tile's copies go out.
+        const bool is_k = warp == kProducerWarp;
+        const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
+        uint64_t* full = is_k ? k_full : v_full;
+        uint64_t* empty = is_k ? k_empty : v_empty;
+        uint8_t* base = is_k ? sK : sV;
         const uint64_t pol = l2_policy_evict_last();     // K/V tiles are re-read by the head's other q-tiles
         if (lane == 0) {
-            tma_prefetch_desc(&tm_q);
-            tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
-            mbar_arrive_expect_tx(q_full, C::kOpBytes);
+            tma_prefetch_desc(tm);
+            if (is_k) {
+                tma_prefetch_desc(&tm_q);
+                mbar_arrive_expect_tx(q_full, C::kOpBytes);
 #pragma unroll
-            for (int c = 0; c < C::kChunks; ++c)
-                tma_load_3d(sQ + c * C::kChunkBytes, &tm_q, q_full, c * 64, h, q0, pol);
+                for (int c = 0; c < C::kChunks; ++c)
+                    tma_load_3d(sQ + c * C::kChunkBytes, &tm_q, q_full, c * 64, h, q0, pol);
+            }
         }
         const int br = p.box_rows;
         const int64_t tbase = static_cast<int64_t>(b) * p.max_blocks;
-        int k_last = -1, v_last = -1;     // last tiles whose K / V copies were issued
-        // Block ids of a tile: lane i holds the physical block of the tile's i-th box.  The ids of
-        // tile j+1 are loaded while tile j's copies are issued, so the table read never stalls a tile.
         auto load_ids = [&](int j) -> int {
             const int key0 = j * kTile;
             const int nbox = (min(kTile, kv_len - key0) + br - 1) / br;
@@ -217,45 +224,31 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             return bid;
         };
+        int last = -1;                                   // last tile whose copies this warp issued
         int bid = load_ids(0);
         for (int j = 0; j < n_tiles; ++j) {
             const int st = j & 1;
             const int key0 = j * kTile;
-            const int nkeys = min(kTile, kv_len - key0);
-            const int nbox = (nkeys + br - 1) / br;
+            const int nbox = (min(kTile, kv_len - key0) + br - 1) / br;
             const int bid_next = load_ids(j + 1);
+            const int box = lane / C::kChunks, chunk = lane % C::kChunks;
+            const int my_bid = __shfl_sync(0xffffffffu, bid, box);
             const uint32_t bytes = static_cast<uint32_t>(nbox * br * 128 * C::kChunks);
-            // Each lane issues its own boxes: the copies of a tile go out in parallel.
-            const int row = bid * p.bs + (key0 + lane * br) % p.bs;
-            // K tile: its stage frees as soon as S of the tile two back has been computed
-            if (!mbar_wait(&k_empty[st], ((j >> 1) & 1) ^ 1)) { abort_now(); break; }
+            if (!mbar_wait(&empty[st], ((j >> 1) & 1) ^ 1)) { abort_now(); break; }
             if (info[2]) break;
-            if (lane == 0) mbar_arrive_expect_tx(&k_full[st], bytes);
+            if (lane == 0) mbar_arrive_expect_tx(&full[st], bytes);
             __syncwarp();
-            if (lane < nbox) {
-                uint8_t* dk = sK + st * C::kOpBytes + lane * br * 128;
-#pragma unroll
-                for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_3d(dk + c * C::kChunkBytes, &tm_k, &k_full[st], c * 64, h, row, pol);
+            if (box < nbox) {
+                const int key = key0 + box * br;
+                tma_load_3d(base + st * C::kOpBytes + chunk * C::kChunkBytes + box * br * 128, tm, &full[st],
+                            chunk * 64, h, my_bid * p.bs + key % p.bs, pol);
             }
-            k_last = j;
-            // V tile: its stage frees when P.V of the tile two back has completed
-            if (!mbar_wait(&v_empty[st], ((j >> 1) & 1) ^ 1)) { abort_now(); break; }
-            if (lane == 0) mbar_arrive_expect_tx(&v_full[st], bytes);
-            __syncwarp();
-            if (lane < nbox) {
-                uint8_t* dv = sV + st * C::kOpBytes + lane * br * 128;
-#pragma unroll
-                for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_3d(dv + c * C::kChunkBytes, &tm_v, &v_full[st], c * 64, h, row, pol);
-            }
-            v_last = j;
+            last = j;
             bid = bid_next;
         }
         if (info[2]) {
-            // unwind: let the copies this warp issued into each stage land
-            for (int j = max(0, k_last - 1); j <= k_last; ++j) (void)mbar_wait(&k_full[j & 1], (j >> 1) & 1);
-            for (int j = max(0, v_last - 1); j <= v_last; ++j) (void)mbar_wait(&v_full[j & 1], (j >> 1) & 1);
+            // unwind: let the copies this warp issued land
+            for (int j = max(0, last - 1); j <= last; ++j) (void)mbar_wait(&full[j & 1], (j >> 1) & 1);
         }
     } else if (warp == kMmaWarp) {
         // ======================================================= MMA issuer
