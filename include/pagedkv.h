@@ -164,6 +164,9 @@ pa_status pa_alloc_pack(const pa_alloc* a, const int64_t* reqs, int32_t n, int32
 
 /* Counters (see pa_alloc_stats_t). */
 pa_status pa_alloc_stats(const pa_alloc* a, pa_alloc_stats_t* out);
+/* *out = blocks a take can use now: the free list plus the prefix cache's
+ * parked blocks.  O(1).  Errors: INVALID_ARG. */
+pa_status pa_alloc_available(const pa_alloc* a, int64_t* out);
 /* *out = refcount of physical block `block`.  Errors: INVALID_ARG. */
 pa_status pa_alloc_refcount(const pa_alloc* a, int32_t block, int32_t* out);
 /* Copy the free list (bottom to top; the next pop takes the last entry).

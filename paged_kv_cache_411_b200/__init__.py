@@ -114,6 +114,11 @@ class BlockAllocator:
         check(lib().pa_alloc_stats(self._h, byref(s)))
         return s.as_dict()
 
+    def available(self) -> int:
+        n = c_int64(0)
+        check(lib().pa_alloc_available(self._h, byref(n)))
+        return n.value
+
     def refcount(self, block: int):
         n = c_int32(0)
         st = lib().pa_alloc_refcount(self._h, block, byref(n))

@@ -112,6 +112,7 @@ SIGNATURES = {
     "pa_alloc_slots": (c_int32, [_P, c_int64, c_int32, c_int32, _I64P]),
     "pa_alloc_pack": (c_int32, [_P, _I64P, c_int32, c_int32, _I32P, _I32P]),
     "pa_alloc_stats": (c_int32, [_P, POINTER(AllocStats)]),
+    "pa_alloc_available": (c_int32, [_P, _I64P]),
     "pa_alloc_refcount": (c_int32, [_P, c_int32, _I32P]),
     "pa_alloc_free_list": (c_int32, [_P, _I32P, c_int32, _I32P]),
     "pa_alloc_allocate_cached": (c_int32, [_P, c_int64, _I32P, c_int32, _I32P]),

@@ -346,6 +346,12 @@ pa_status pa_alloc_stats(const pa_alloc* a, pa_alloc_stats_t* out) {
     return PA_OK;
 }
 
+pa_status pa_alloc_available(const pa_alloc* a, int64_t* out) {
+    if (!a || !out) return fail(PA_ERR_INVALID_ARG, "pa_alloc_available: NULL argument");
+    *out = a->available();
+    return PA_OK;
+}
+
 pa_status pa_alloc_refcount(const pa_alloc* a, int32_t block, int32_t* out) {
     if (!a || !out || block < 0 || block >= a->num_blocks)
         return fail(PA_ERR_INVALID_ARG, "pa_alloc_refcount: bad block %d", block);

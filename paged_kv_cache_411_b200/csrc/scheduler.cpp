@@ -68,11 +68,9 @@ struct pa_sched {
     int64_t steps = 0, preemptions = 0, finished = 0, prefill_tokens = 0, decode_tokens = 0;
 
     int64_t available() const {
-        pa_alloc_stats_t s;
-        pa_cache_stats_t c;
-        pa_alloc_stats(alloc, &s);
-        pa_alloc_cache_stats(alloc, &c);
-        return static_cast<int64_t>(s.num_free) + c.evictable_blocks;
+        int64_t n = 0;
+        pa_alloc_available(alloc, &n);
+        return n;
     }
     int32_t kv_len(int64_t r) const {
         int32_t n = 0;

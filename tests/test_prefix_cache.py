@@ -112,3 +112,12 @@ def test_prefix_cache_errors():
     assert ca.allocate_cached(2, [1, 2, 9, 9, 9, 9, 9]) == (pk.PA_ERR_OOM, 0)
     assert ca.stats()["oom_count"] == 1 and ca.cache_stats()["cached_blocks"] == 1
     assert ca.allocate_cached(3, []) == (pk.PA_OK, 0)
+
+
+def test_available_counts_free_and_parked_blocks():
+    a = pk.BlockAllocator(6, 2)
+    assert a.available() == 6
+    assert a.allocate_cached(1, [1, 2, 3, 4, 5]) == (pk.PA_OK, 0)     # 3 blocks, 2 registered
+    assert a.available() == 3
+    a.free(1)                                                          # 2 parked, 1 freed
+    assert a.available() == 6 and len(a.evictable_list()) == 2 and len(a.free_list()) == 4
