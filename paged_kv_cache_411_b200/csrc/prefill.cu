@@ -331,20 +331,25 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const uint32_t sa = lane_base + C::kColS + (j & 1) * kTile + g * 64;
             float sv[64];
             {
-                float v0[32], v1[32];
-                tmem_ld_32cols(sa, v0);
-                tmem_ld_32cols(sa + 32, v1);
+                uint32_t r0[32], r1[32];                  // both loads in flight, one wait
+                tmem_ld_32cols_nowait(sa, r0);
+                tmem_ld_32cols_nowait(sa + 32, r1);
+                tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) { sv[i] = v0[i]; sv[32 + i] = v1[i]; }
+                for (int i = 0; i < 32; ++i) { sv[i] = __uint_as_float(r0[i]); sv[32 + i] = __uint_as_float(r1[i]); }
             }
             if (diag) {
 #pragma unroll
                 for (int i = 0; i < 64; ++i)
                     if (key0 + g * 64 + i > row_pos) sv[i] = -INFINITY;
             }
-            float mx = sv[0];
+            float mx8[8];
 #pragma unroll
-            for (int i = 1; i < 64; ++i) mx = fmaxf(mx, sv[i]);
+            for (int k = 0; k < 8; ++k) mx8[k] = sv[k];
+#pragma unroll
+            for (int i = 8; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
+            float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             // raw scores: scale > 0 keeps the order, so the max is taken before scaling
             float* rm = red + (j & 1) * 256;
             rm[g * 128 + r] = mx;
@@ -356,20 +361,25 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const float m_use = m_new == -INFINITY ? 0.f : m_new;
             const float alpha = exp2f(m - m_use);
             if (!(ok = mbar_wait(p_empty, (j & 1) ^ 1))) break;
-            float rs = 0.f;
+            // P = 2^(s*scale*log2e - m) computed two at a time in fp16 (P is stored in fp16 for the
+            // P.V MMA anyway); the row sum adds exactly the fp16 values that MMA will use.
+            float rs4[4] = {0.f, 0.f, 0.f, 0.f};
             uint8_t* prow = sP + g * C::kChunkBytes + r * 128;
 #pragma unroll
             for (int u = 0; u < 8; ++u) {                     // 8 keys = one 16-byte unit of P
                 uint32_t pk[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const float p0 = exp2f(fmaf(sv[8 * u + 2 * i], qs, -m_use));
-                    const float p1 = exp2f(fmaf(sv[8 * u + 2 * i + 1], qs, -m_use));
-                    rs += p0 + p1;
-                    pk[i] = f2_to_h2(p0, p1);
+                    const __half2 x = __floats2half2_rn(fmaf(sv[8 * u + 2 * i], qs, -m_use),
+                                                        fmaf(sv[8 * u + 2 * i + 1], qs, -m_use));
+                    const __half2 e = h2exp2(x);
+                    const float2 ef = __half22float2(e);
+                    rs4[i] += ef.x + ef.y;
+                    pk[i] = *reinterpret_cast<const uint32_t*>(&e);
                 }
                 st_shared_u4(prow + ((u ^ (r & 7)) * 16), make_uint4(pk[0], pk[1], pk[2], pk[3]));
             }
+            const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_empty[j & 1]);

@@ -152,3 +152,18 @@ def test_prefill_device_checks(cuda_ready):
                                      err_flag=err)
     torch.cuda.synchronize()
     assert int(err.item()) & pk.PA_DEVCHK_SEQ_LEN
+
+
+@pytest.mark.parametrize("qmul", [4.0, 8.0])
+def test_prefill_sharp_softmax(cuda_ready, qmul):
+    """Sharper score distributions (q scaled up): the exponent arguments span a wide range, which
+    exercises the fp16 exp2 of P; the output must still be within the tolerance."""
+    H, D, bs = 4, 128, 16
+    case = make_case(17, H, D, bs, [(300, 200), (0, 129)])
+    case["q"] = (case["q"].astype(np.float32) * qmul).astype(np.float16)
+    case["dev"]["q"] = torch.from_numpy(case["q"]).cuda()
+    scale = 1 / np.sqrt(D)
+    out = run_prefill(case, scale).float().cpu().numpy()
+    ref = oracle_prefill(case, bs, scale)
+    diff = np.abs(out - ref)
+    assert diff.max() <= TOL, f"max abs error {diff.max():.3g}"
