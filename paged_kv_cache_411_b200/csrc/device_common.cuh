@@ -114,6 +114,15 @@ __device__ __forceinline__ uint32_t f2_to_h2(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// acc + lo(h2) + hi(h2): PTX's mixed-precision add (sm_100+) widens each fp16 half exactly and adds
+// it in fp32, so a sum of fp16 values costs no separate conversion.
+__device__ __forceinline__ float add_h2_f32(float acc, uint32_t h2) {
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tadd.rn.f32.f16 %0, lo, %0;\n\tadd.rn.f32.f16 %0, hi, %0;\n\t}"
+        : "+f"(acc)
+        : "r"(h2));
+    return acc;
+}
+
 }  // namespace pagedkv
 
 namespace pagedkv {
@@ -186,6 +195,21 @@ __device__ __forceinline__ void tmem_ld_32cols_nowait(uint32_t taddr, uint32_t (
           "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
 }
+
+// Writes 32 consecutive fp32 columns of this thread's TMEM lane (same lane rule as the loads); the
+// caller issues tmem_wait_st() before signalling that the columns are ready.
+__device__ __forceinline__ void tmem_st_32cols(uint32_t taddr, const float (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+        ::"r"(taddr), "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]),
+          "f"(v[8]), "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15]),
+          "f"(v[16]), "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]),
+          "f"(v[24]), "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // 16 consecutive fp32 columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_ld_16cols(uint32_t taddr, float (&v)[16]) {

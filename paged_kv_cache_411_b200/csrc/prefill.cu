@@ -17,16 +17,23 @@
 //     canonical UMMA layout; each lane issues one box, so a tile is one TMA
 //     instruction, and the next tile's block ids are read a tile ahead;
 //   * warp 9 (one elected thread) issues tcgen05.mma: S = Q K^T (A and B
-//     K-major) into a double-buffered fp32 TMEM tile, and O_j = P_j V_j (B
-//     MN-major straight from the V tile) into a second double-buffered TMEM
-//     tile; completions are signalled with tcgen05.commit on mbarriers;
-//   * warps 0-7 (two threads per query row = per TMEM lane, each owning half
-//     of the columns) read S with tcgen05.ld, apply the causal mask on the
-//     diagonal tiles, agree on the row max through shared memory, run the
-//     online softmax in fp32 (exp2 of prescaled logits), write P as fp16 into
-//     shared memory in the swizzled K-major layout the next MMA reads, and
-//     fold O_j into a register accumulator with the running rescale one tile
-//     behind, so the MMA of tile j+1 overlaps the softmax of tile j.
+//     K-major) into a double-buffered fp32 TMEM tile, and P V (B MN-major
+//     straight from the V tile) accumulated in TMEM across all key tiles as two
+//     partial outputs, O_0 over the first 64 keys of every tile and O_1 over the
+//     last 64; completions are signalled with tcgen05.commit on mbarriers;
+//   * warps 0-7 (two threads per query row = per TMEM lane; thread g of a row
+//     owns key columns g*64 .. g*64+63 of every tile and so the partial output
+//     O_g) read S with tcgen05.ld, apply the causal mask on the diagonal tiles
+//     and run the online softmax of their half on their own: each keeps its own
+//     running max m_g and sum l_g, and P = 2^(s*scale*log2e - m_g) is written
+//     as fp16 into shared memory in the swizzled K-major layout the next MMA
+//     reads.  m_g only moves when a tile's max exceeds it by more than
+//     kRescaleLog2 (P then stays <= 2^kRescaleLog2, exact in fp16 up to its
+//     11-bit mantissa); when it moves, the warp rescales its rows of O_g in
+//     TMEM (after the previous P V has completed) before the next P V adds to
+//     it.  The two halves of a row are merged once, after the last tile:
+//     O = (O_0 2^(m_0-M) + O_1 2^(m_1-M)) / (l_0 2^(m_0-M) + l_1 2^(m_1-M)),
+//     M = max(m_0, m_1).  The MMA of tile j+1 overlaps the softmax of tile j.
 // Keys past the tile's last query position are masked; rows of V past the
 // sequence end are zeroed before P.V so stale or poisoned pool rows never
 // reach the MMA.  Every wait is bounded; on a timeout the CTA records
@@ -40,12 +47,15 @@ namespace pagedkv {
 namespace {
 
 constexpr int kTile = 128;
-constexpr int kSoftmaxWarps = 8;          // two warpgroups: each owns half of the S / O columns
+constexpr int kSoftmaxWarps = 8;          // two warpgroups: each owns half of the key columns of S
 constexpr int kProducerWarp = 8;          // Q and K tiles
 constexpr int kMmaWarp = 9;
 constexpr int kProducerVWarp = 10;        // V tiles
 constexpr int kThreadsP = 11 * 32;
 constexpr float kLog2eP = 1.4426950408889634f;
+// A thread's running max (log2 domain) is raised only when a tile's max exceeds it by more than this;
+// P <= 2^kRescaleLog2 = 256 is exact enough in fp16 and far from its overflow.
+constexpr float kRescaleLog2 = 8.f;
 
 struct PrefillParams {
     __half* out;
@@ -68,16 +78,16 @@ struct PCfg {
     static constexpr size_t kOffV = kOffK + size_t(kStages) * kOpBytes;
     static constexpr size_t kOffP = kOffV + size_t(kStages) * kOpBytes;
     static constexpr size_t kOffBar = kOffP + 2 * kChunkBytes;    // P: 128 rows x 128 keys fp16
-    static constexpr int kNumBars = 23;
+    static constexpr int kNumBars = 17;
     static constexpr size_t kOffSlot = kOffBar + kNumBars * 8;
-    static constexpr size_t kOffRed = kOffSlot + 64;                 // row-max exchange [2][2][128] + row sums [2][128]
+    static constexpr size_t kOffRed = kOffSlot + 64;                 // final exchange: maxes [2][128], sums [2][128]
     // Every CTA takes all 512 TMEM columns, so the request is kept above half the SM's shared
     // memory: one CTA per SM, and tcgen05.alloc never has to wait for a neighbour.
-    static constexpr size_t kSmemUsed = kOffRed + 6 * 128 * 4 + 1024;
+    static constexpr size_t kSmemUsed = kOffRed + 4 * 128 * 4 + 1024;
     static constexpr size_t kSmemBytes = kSmemUsed > 120 * 1024 ? kSmemUsed : 120 * 1024;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColS = 0;                          // S buffers: columns 0 and 128
-    static constexpr uint32_t kColO = 256;                        // O buffers: 256 and 256 + D
+    static constexpr uint32_t kColO = 256;                        // O_0 at 256, O_1 at 256 + D
 };
 
 __device__ __forceinline__ void st_shared_u4(void* p, uint4 v) {
@@ -102,16 +112,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint64_t* k_full = bars + 1;     // [2]
     uint64_t* v_full = bars + 3;     // [2]
     uint64_t* k_empty = bars + 5;    // [2] released by the S MMA
-    uint64_t* v_empty = bars + 21;   // [2] released by the P.V MMA
+    uint64_t* v_empty = bars + 15;   // [2] released by the P.V MMA
     uint64_t* s_full = bars + 7;     // [2]
     uint64_t* s_empty = bars + 9;    // [2]
     uint64_t* p_full = bars + 11;
-    uint64_t* p_empty = bars + 12;
-    uint64_t* o_full = bars + 13;    // [2]
-    uint64_t* o_empty = bars + 15;   // [2]
-    uint64_t* drain = bars + 17;
-    uint64_t* red_bar = bars + 18;   // [2] row-max exchange between the two softmax warpgroups
-    uint64_t* sum_bar = bars + 20;   // final row-sum exchange
+    uint64_t* pv_done = bars + 12;   // phase j completes when the P.V of tile j has (P free, O_g readable)
+    uint64_t* drain = bars + 13;
+    uint64_t* sum_bar = bars + 14;   // final (max, sum) exchange between the two halves of a row
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffSlot);
     volatile int* info = reinterpret_cast<volatile int*>(smem + C::kOffSlot + 16);   // b, qt, abort
 
@@ -151,14 +158,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&v_empty[i], 1);
             mbar_init(&s_full[i], 1);
             mbar_init(&s_empty[i], kSoftmaxWarps);
-            mbar_init(&o_full[i], 1);
-            mbar_init(&o_empty[i], kSoftmaxWarps);
         }
         mbar_init(p_full, kSoftmaxWarps);
-        mbar_init(p_empty, 1);
+        mbar_init(pv_done, 1);
         mbar_init(drain, 1);
-        mbar_init(&red_bar[0], kSoftmaxWarps);
-        mbar_init(&red_bar[1], kSoftmaxWarps);
         mbar_init(sum_bar, kSoftmaxWarps);
         mbar_init_fence();
     }
@@ -280,19 +283,19 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const int st = j & 1;
                 if (!(ok = mbar_wait(p_full, j & 1))) break;
                 if (!(ok = mbar_wait(&v_full[st], (j >> 1) & 1))) break;
-                if (!(ok = mbar_wait(&o_empty[j & 1], ((j >> 1) & 1) ^ 1))) break;
                 if (info[2]) { ok = false; break; }
                 tc_fence_after_sync();
-                const uint32_t d = tmem + C::kColO + (j & 1) * D;
                 const uint32_t vb = aV + st * C::kOpBytes;
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk) {
+                    // keys 0-63 of the tile add to O_0, keys 64-127 to O_1; tile 0 starts both
+                    const uint32_t d = tmem + C::kColO + (kk >> 2) * D;
                     const uint32_t poff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
                     umma_f16_ss(d, umma_desc_sw128(aP + poff, 16, 1024),
-                                umma_desc_sw128(vb + kk * 16 * 128, C::kChunkBytes, 1024), idesc_pv, kk > 0);
+                                umma_desc_sw128(vb + kk * 16 * 128, C::kChunkBytes, 1024), idesc_pv,
+                                j > 0 || (kk & 3) != 0);
                 }
-                umma_commit(&o_full[j & 1]);
-                umma_commit(p_empty);
+                umma_commit(pv_done);
                 umma_commit(&v_empty[st]);
             }
             if (!ok) {
@@ -305,9 +308,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         __syncwarp();
     } else {
         // ======================================================= softmax warps
-        // Thread (warpgroup g, row r): row r of the tile (TMEM lane r), columns g*64 .. g*64+63 of S
-        // and g*D/2 .. (g+1)*D/2-1 of O.  The two threads of a row agree on the running max through
-        // shared memory once per tile; each keeps a partial row sum, added at the end.
+        // Thread (warpgroup g, row r): row r of the tile (TMEM lane r), key columns g*64 .. g*64+63 of
+        // every S tile, and the partial output O_g of those keys (all D columns of row r).
         const int g = warp >> 2;
         const int r = (warp & 3) * 32 + lane;
         const int row_in_req = qt * kTile + r;
@@ -315,14 +317,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int row_pos = min(ctx + row_in_req, kv_len - 1);
         const int tile_pos0 = ctx + qt * kTile;          // smallest query position in the tile
         const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-        constexpr int DH = D / 2;
-        float* red = reinterpret_cast<float*>(smem + C::kOffRed);    // [parity][g][row], then sums [g][row]
+        const uint32_t o_mine = lane_base + C::kColO + g * D;
         const float qs = p.qscale;
-        float acc[DH];
-#pragma unroll
-        for (int i = 0; i < DH; ++i) acc[i] = 0.f;
-        float m = -INFINITY, l = 0.f, alpha_prev = 0.f;
+        float m = -INFINITY, l = 0.f;                    // log2-domain running max and sum of this half
         bool ok = true;
+        uint8_t* prow = sP + g * C::kChunkBytes + r * 128;
         for (int j = 0; j < n_tiles && ok; ++j) {
             if (!(ok = mbar_wait(&s_full[j & 1], (j >> 1) & 1))) break;
             tc_fence_after_sync();
@@ -338,6 +337,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
                 for (int i = 0; i < 32; ++i) { sv[i] = __uint_as_float(r0[i]); sv[32 + i] = __uint_as_float(r1[i]); }
             }
+            // S is in registers: the buffer can take the tile after next
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[j & 1]);
             if (diag) {
 #pragma unroll
                 for (int i = 0; i < 64; ++i)
@@ -348,41 +351,43 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             for (int k = 0; k < 8; ++k) mx8[k] = sv[k];
 #pragma unroll
             for (int i = 8; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
-            float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             // raw scores: scale > 0 keeps the order, so the max is taken before scaling
-            float* rm = red + (j & 1) * 256;
-            rm[g * 128 + r] = mx;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&red_bar[j & 1]);
-            if (!(ok = mbar_wait(&red_bar[j & 1], (j >> 1) & 1))) break;
-            mx = fmaxf(mx, rm[(g ^ 1) * 128 + r]) * qs;
-            const float m_new = fmaxf(m, mx);
-            const float m_use = m_new == -INFINITY ? 0.f : m_new;
-            const float alpha = exp2f(m - m_use);
-            if (!(ok = mbar_wait(p_empty, (j & 1) ^ 1))) break;
-            // P = 2^(s*scale*log2e - m) computed two at a time in fp16 (P is stored in fp16 for the
-            // P.V MMA anyway); the row sum adds exactly the fp16 values that MMA will use.
-            float rs4[4] = {0.f, 0.f, 0.f, 0.f};
-            uint8_t* prow = sP + g * C::kChunkBytes + r * 128;
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {                     // 8 keys = one 16-byte unit of P
-                uint32_t pk[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const __half2 x = __floats2half2_rn(fmaf(sv[8 * u + 2 * i], qs, -m_use),
-                                                        fmaf(sv[8 * u + 2 * i + 1], qs, -m_use));
-                    const __half2 e = h2exp2(x);
-                    const float2 ef = __half22float2(e);
-                    rs4[i] += ef.x + ef.y;
-                    pk[i] = *reinterpret_cast<const uint32_t*>(&e);
-                }
-                st_shared_u4(prow + ((u ^ (r & 7)) * 16), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * qs;
+            float alpha = 1.f;
+            const bool raise = mx > m + kRescaleLog2;                // false while both are -inf
+            if (raise) {
+                alpha = exp2f(m - mx);                               // 0 when m is still -inf
+                m = mx;
             }
-            const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_empty[j & 1]);
+            const float m_use = m == -INFINITY ? 0.f : m;
+            uint32_t pk[32];
+            float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const float p0 = exp2f(fmaf(sv[2 * i], qs, -m_use));
+                const float p1 = exp2f(fmaf(sv[2 * i + 1], qs, -m_use));
+                pk[i] = f2_to_h2(p0, p1);
+                rs4[i & 3] = add_h2_f32(rs4[i & 3], pk[i]);   // the fp16 values the P.V MMA adds
+            }
+            l = fmaf(l, alpha, (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
+            // the P.V of tile j-1 has read P and added to O_g before either is touched
+            if (!(ok = mbar_wait(pv_done, (j & 1) ^ 1))) break;
+            if (j > 0 && __any_sync(0xffffffffu, raise)) {
+                tc_fence_after_sync();
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    float v[32];
+                    tmem_ld_32cols(o_mine + c * 32, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] *= alpha;
+                    tmem_st_32cols(o_mine + c * 32, v);
+                }
+                tmem_wait_st();
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)                               // 8 keys = one 16-byte unit of P
+                st_shared_u4(prow + ((u ^ (r & 7)) * 16), make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]));
             if (j == n_tiles - 1 && kv_len < key0 + kTile) {
                 // rows of V past the sequence end may hold anything: zero them before P.V reads them
                 if (!(ok = mbar_wait(&v_full[j & 1], (j >> 1) & 1))) break;
@@ -395,63 +400,49 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             st_shared_u4(vrow + c * C::kChunkBytes + (g * 4 + u) * 16, make_uint4(0, 0, 0, 0));
                 }
             }
+            tc_fence_before_sync();
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(p_full);
-            l = fmaf(l, alpha, rs);
-            if (j > 0) {
-                const int jp = j - 1;
-                if (!(ok = mbar_wait(&o_full[jp & 1], (jp >> 1) & 1))) break;
-                tc_fence_after_sync();
-                const uint32_t oa = lane_base + C::kColO + (jp & 1) * D + g * DH;
-#pragma unroll
-                for (int c = 0; c < DH / 32; ++c) {
-                    float v[32];
-                    tmem_ld_32cols(oa + c * 32, v);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[c * 32 + i] = fmaf(acc[c * 32 + i], alpha_prev, v[i]);
-                }
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&o_empty[jp & 1]);
-            }
-            alpha_prev = alpha;
-            m = m_new;
             if (info[2]) ok = false;
         }
-        if (ok) {
-            const int jp = n_tiles - 1;
-            ok = mbar_wait(&o_full[jp & 1], (jp >> 1) & 1);
-            if (ok) {
-                tc_fence_after_sync();
-                const uint32_t oa = lane_base + C::kColO + (jp & 1) * D + g * DH;
-#pragma unroll
-                for (int c = 0; c < DH / 32; ++c) {
-                    float v[32];
-                    tmem_ld_32cols(oa + c * 32, v);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[c * 32 + i] = fmaf(acc[c * 32 + i], alpha_prev, v[i]);
-                }
-            }
-        }
-        // both threads of a row add their partial sums (every softmax thread reaches this barrier)
-        float* rsum = red + 512;
-        rsum[g * 128 + r] = l;
+        // merge the two halves of the row (every softmax thread reaches this barrier)
+        float* red = reinterpret_cast<float*>(smem + C::kOffRed);    // maxes [g][row], then sums [g][row]
+        red[g * 128 + r] = m;
+        red[256 + g * 128 + r] = l;
         __syncwarp();
         if (lane == 0) mbar_arrive(sum_bar);
         if (ok) ok = mbar_wait(sum_bar, 0);
-        l += rsum[(g ^ 1) * 128 + r];
-        if (ok && row_valid) {
-            const float inv = 1.f / l;
+        if (ok) ok = mbar_wait(pv_done, (n_tiles - 1) & 1);        // the last P.V has landed in O_0, O_1
+        if (ok) {
+            tc_fence_after_sync();
+            const float m0 = red[r], m1 = red[128 + r];
+            const float mm = fmaxf(m0, m1);
+            const float c0 = exp2f(m0 - mm), c1 = exp2f(m1 - mm);    // a half that saw no key: 0
+            const float inv = 1.f / (red[256 + r] * c0 + red[384 + r] * c1);
+            const float s0 = c0 * inv, s1 = c1 * inv;
+            constexpr int DH = D / 2;                                // this thread writes columns g*DH ..
             __half* orow = p.out + (static_cast<int64_t>(q0 + r) * p.H + h) * D + g * DH;
+#pragma unroll 1
+            for (int c = 0; c < DH / 32; ++c) {
+                uint32_t a0[32], a1[32];
+                tmem_ld_32cols_nowait(lane_base + C::kColO + g * DH + c * 32, a0);
+                tmem_ld_32cols_nowait(lane_base + C::kColO + D + g * DH + c * 32, a1);
+                tmem_wait_ld();
+                if (row_valid) {
 #pragma unroll
-            for (int c = 0; c < DH / 8; ++c) {
-                uint4 o;
-                o.x = f2_to_h2(acc[8 * c + 0] * inv, acc[8 * c + 1] * inv);
-                o.y = f2_to_h2(acc[8 * c + 2] * inv, acc[8 * c + 3] * inv);
-                o.z = f2_to_h2(acc[8 * c + 4] * inv, acc[8 * c + 5] * inv);
-                o.w = f2_to_h2(acc[8 * c + 6] * inv, acc[8 * c + 7] * inv);
-                *reinterpret_cast<uint4*>(orow + 8 * c) = o;
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 o;
+                        uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int i = 8 * q + 2 * e;
+                            ow[e] = f2_to_h2(__uint_as_float(a0[i]) * s0 + __uint_as_float(a1[i]) * s1,
+                                             __uint_as_float(a0[i + 1]) * s0 + __uint_as_float(a1[i + 1]) * s1);
+                        }
+                        *reinterpret_cast<uint4*>(orow + c * 32 + 8 * q) = o;
+                    }
+                }
             }
         }
         if (!ok) abort_now();

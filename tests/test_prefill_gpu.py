@@ -154,7 +154,7 @@ def test_prefill_device_checks(cuda_ready):
     assert int(err.item()) & pk.PA_DEVCHK_SEQ_LEN
 
 
-@pytest.mark.parametrize("qmul", [4.0, 8.0])
+@pytest.mark.parametrize("qmul", [4.0, 8.0, 16.0])
 def test_prefill_sharp_softmax(cuda_ready, qmul):
     """Sharper score distributions (q scaled up): the exponent arguments span a wide range, which
     exercises the fp16 exp2 of P; the output must still be within the tolerance."""
