@@ -10,13 +10,14 @@
 //
 // One CTA computes one tile of 128 query rows x one head (FlashAttention
 // order, online softmax over 128-key tiles):
-//   * warps 8 and 10 (producers) load the Q tile once and stream the K and the
-//     V tiles into two-stage rings with TMA: a tile of 128 keys is gathered from
-//     the paged pool with one 3-D box per (physical block, 64-dim chunk) ([box
-//     rows][1 head][64 dims], 128-byte swizzle), landing directly in the
-//     canonical UMMA layout; each lane issues one box, so a tile is one TMA
-//     instruction, and the next tile's block ids are read a tile ahead;
-//   * warp 9 (one elected thread) issues tcgen05.mma: S = Q K^T (A and B
+//   * kIssueWarps K warps and kIssueWarps V warps (producers, from warp 8) load
+//     the Q tile once and stream the K and the V tiles into two-stage rings
+//     with TMA: a tile of 128 keys is gathered from the paged pool with one 3-D
+//     box per (physical block, 64-dim chunk) ([box rows][1 head][64 dims],
+//     128-byte swizzle), landing directly in the canonical UMMA layout; the
+//     boxes are dealt to the lanes of the operand's warps, one each, and the
+//     next tile's block ids are read a tile ahead;
+//   * the last warp (one elected thread) issues tcgen05.mma: S = Q K^T (A and B
 //     K-major) into a double-buffered fp32 TMEM tile, and P V (B MN-major
 //     straight from the V tile) accumulated in TMEM across all key tiles as two
 //     partial outputs, O_0 over the first 64 keys of every tile and O_1 over the
@@ -48,10 +49,11 @@ namespace {
 
 constexpr int kTile = 128;
 constexpr int kSoftmaxWarps = 8;          // two warpgroups: each owns half of the key columns of S
-constexpr int kProducerWarp = 8;          // Q and K tiles
-constexpr int kMmaWarp = 9;
-constexpr int kProducerVWarp = 10;        // V tiles
-constexpr int kThreadsP = 11 * 32;
+constexpr int kIssueWarps = 2;                        // TMA-issuing warps per operand (K, V)
+constexpr int kFirstKWarp = 8;                        // K warps (the first also loads Q)
+constexpr int kFirstVWarp = kFirstKWarp + kIssueWarps;
+constexpr int kMmaWarp = kFirstVWarp + kIssueWarps;
+constexpr int kThreadsP = (kMmaWarp + 1) * 32;
 constexpr float kLog2eP = 1.4426950408889634f;
 // A thread's running max (log2 domain) is raised only when a tile's max exceeds it by more than this;
 // P <= 2^kRescaleLog2 = 256 is exact enough in fp16 and far from its overflow.
@@ -152,8 +154,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         info[2] = 0;
         mbar_init(q_full, 1);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&k_full[i], 1);
-            mbar_init(&v_full[i], 1);
+            mbar_init(&k_full[i], kIssueWarps);
+            mbar_init(&v_full[i], kIssueWarps);
             mbar_init(&k_empty[i], 1);
             mbar_init(&v_empty[i], 1);
             mbar_init(&s_full[i], 1);
@@ -191,12 +193,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         info[2] = 1;
     };
 
-    if (warp == kProducerWarp || warp == kProducerVWarp) {
-        // ======================================================= TMA producers (K warp, V warp)
-        // A 128-key tile is one box per (physical block, 64-dim chunk): lane L issues box L of the tile,
-        // so a tile goes out as one TMA instruction.  The next tile's block ids are read while the
-        // current tile's copies go out.
-        const bool is_k = warp == kProducerWarp;
+    if (warp >= kFirstKWarp && warp < kMmaWarp) {
+        // ======================================================= TMA producers (K warps, V warps)
+        // A 128-key tile is one box per (physical block, 64-dim chunk).  The boxes of a tile are dealt
+        // round-robin to the operand's kIssueWarps warps, one per lane, so a tile goes out as one TMA
+        // instruction per warp; every warp arrives on the stage's barrier with its own byte count.
+        // Each lane reads the block id of its box of the next tile while the current tile's copies go
+        // out, and checks it only when it uses it, so the read's latency stays off the issue path.
+        const bool is_k = warp < kFirstVWarp;
+        const int wsub = warp - (is_k ? kFirstKWarp : kFirstVWarp);
         const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
         uint64_t* full = is_k ? k_full : v_full;
         uint64_t* empty = is_k ? k_empty : v_empty;
@@ -204,7 +209,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const uint64_t pol = l2_policy_evict_last();     // K/V tiles are re-read by the head's other q-tiles
         if (lane == 0) {
             tma_prefetch_desc(tm);
-            if (is_k) {
+            if (is_k && wsub == 0) {
                 tma_prefetch_desc(&tm_q);
                 mbar_arrive_expect_tx(q_full, C::kOpBytes);
 #pragma unroll
@@ -214,35 +219,31 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         const int br = p.box_rows;
         const int64_t tbase = static_cast<int64_t>(b) * p.max_blocks;
-        auto load_ids = [&](int j) -> int {
-            const int key0 = j * kTile;
-            const int nbox = (min(kTile, kv_len - key0) + br - 1) / br;
-            int bid = 0;
-            if (j < n_tiles && lane < nbox) {
-                bid = p.block_tables[tbase + (key0 + lane * br) / p.bs];
-                if (bid < 0 || bid >= p.num_blocks) {
-                    flag_error(p.err_flag, PA_DEVCHK_BLOCK_ID);
-                    bid = 0;
-                }
-            }
-            return bid;
+        const int my_i = lane * kIssueWarps + wsub;      // this lane's box of every tile
+        const int box = my_i / C::kChunks, chunk = my_i % C::kChunks;
+        auto nbox_of = [&](int j) { return (min(kTile, kv_len - j * kTile) + br - 1) / br; };
+        auto read_id = [&](int j) -> int {               // raw table entry; checked at use
+            return (j < n_tiles && box < nbox_of(j)) ? p.block_tables[tbase + (j * kTile + box * br) / p.bs] : 0;
         };
         int last = -1;                                   // last tile whose copies this warp issued
-        int bid = load_ids(0);
+        int bid = read_id(0);
         for (int j = 0; j < n_tiles; ++j) {
             const int st = j & 1;
-            const int key0 = j * kTile;
-            const int nbox = (min(kTile, kv_len - key0) + br - 1) / br;
-            const int bid_next = load_ids(j + 1);
-            const int box = lane / C::kChunks, chunk = lane % C::kChunks;
-            const int my_bid = __shfl_sync(0xffffffffu, bid, box);
-            const uint32_t bytes = static_cast<uint32_t>(nbox * br * 128 * C::kChunks);
+            const int nbox = nbox_of(j);
+            const int bid_next = read_id(j + 1);
+            const int n_mine = (nbox * C::kChunks - wsub + kIssueWarps - 1) / kIssueWarps;
+            const uint32_t bytes = static_cast<uint32_t>(n_mine * br * 128);
             if (!mbar_wait(&empty[st], ((j >> 1) & 1) ^ 1)) { abort_now(); break; }
             if (info[2]) break;
             if (lane == 0) mbar_arrive_expect_tx(&full[st], bytes);
             __syncwarp();
             if (box < nbox) {
-                const int key = key0 + box * br;
+                int my_bid = bid;
+                if (my_bid < 0 || my_bid >= p.num_blocks) {
+                    flag_error(p.err_flag, PA_DEVCHK_BLOCK_ID);
+                    my_bid = 0;
+                }
+                const int key = j * kTile + box * br;
                 tma_load_3d(base + st * C::kOpBytes + chunk * C::kChunkBytes + box * br * 128, tm, &full[st],
                             chunk * 64, h, my_bid * p.bs + key % p.bs, pol);
             }
