@@ -18,21 +18,23 @@
 //     boxes are dealt to the lanes of the operand's warps, one each, and the
 //     next tile's block ids are read a tile ahead;
 //   * the last warp (one elected thread) issues tcgen05.mma: S = Q K^T (A and B
-//     K-major) into a double-buffered fp32 TMEM tile, and P V (B MN-major
-//     straight from the V tile) accumulated in TMEM across all key tiles as two
-//     partial outputs, O_0 over the first 64 keys of every tile and O_1 over the
-//     last 64; completions are signalled with tcgen05.commit on mbarriers;
+//     K-major) into a double-buffered fp32 TMEM tile, and P V (A = P read from
+//     TMEM, B MN-major straight from the V tile) accumulated in TMEM across all
+//     key tiles as two partial outputs, O_0 over the first 64 keys of every
+//     tile and O_1 over the last 64; completions are signalled with
+//     tcgen05.commit on mbarriers;
 //   * warps 0-7 (two threads per query row = per TMEM lane; thread g of a row
 //     owns key columns g*64 .. g*64+63 of every tile and so the partial output
 //     O_g) read S with tcgen05.ld, apply the causal mask on the diagonal tiles
 //     and run the online softmax of their half on their own: each keeps its own
 //     running max m_g and sum l_g, and P = 2^(s*scale*log2e - m_g) is written
-//     as fp16 into shared memory in the swizzled K-major layout the next MMA
-//     reads.  m_g only moves when a tile's max exceeds it by more than
-//     kRescaleLog2 (P then stays <= 2^kRescaleLog2, exact in fp16 up to its
-//     11-bit mantissa); when it moves, the warp rescales its rows of O_g in
-//     TMEM (after the previous P V has completed) before the next P V adds to
-//     it.  The two halves of a row are merged once, after the last tile:
+//     as fp16 pairs over the first half of the thread's own S columns in TMEM,
+//     where the P V MMA reads it (shared memory carries only Q, K and V).
+//     m_g only moves when a tile's max exceeds it by more than kRescaleLog2
+//     (P then stays <= 2^kRescaleLog2, exact in fp16 up to its 11-bit
+//     mantissa); when it moves, the warp rescales its rows of O_g in TMEM
+//     (after the previous P V has completed) before the next P V adds to it.
+//     The two halves of a row are merged once, after the last tile:
 //     O = (O_0 2^(m_0-M) + O_1 2^(m_1-M)) / (l_0 2^(m_0-M) + l_1 2^(m_1-M)),
 //     M = max(m_0, m_1).  The MMA of tile j+1 overlaps the softmax of tile j.
 // Keys past the tile's last query position are masked; rows of V past the
@@ -78,8 +80,7 @@ struct PCfg {
     static constexpr size_t kOffQ = 0;
     static constexpr size_t kOffK = kOffQ + kOpBytes;
     static constexpr size_t kOffV = kOffK + size_t(kStages) * kOpBytes;
-    static constexpr size_t kOffP = kOffV + size_t(kStages) * kOpBytes;
-    static constexpr size_t kOffBar = kOffP + 2 * kChunkBytes;    // P: 128 rows x 128 keys fp16
+    static constexpr size_t kOffBar = kOffV + size_t(kStages) * kOpBytes;
     static constexpr int kNumBars = 17;
     static constexpr size_t kOffSlot = kOffBar + kNumBars * 8;
     static constexpr size_t kOffRed = kOffSlot + 64;                 // final exchange: maxes [2][128], sums [2][128]
@@ -108,7 +109,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint8_t* sQ = smem + C::kOffQ;
     uint8_t* sK = smem + C::kOffK;
     uint8_t* sV = smem + C::kOffV;
-    uint8_t* sP = smem + C::kOffP;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* q_full = bars + 0;
     uint64_t* k_full = bars + 1;     // [2]
@@ -116,9 +116,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint64_t* k_empty = bars + 5;    // [2] released by the S MMA
     uint64_t* v_empty = bars + 15;   // [2] released by the P.V MMA
     uint64_t* s_full = bars + 7;     // [2]
-    uint64_t* s_empty = bars + 9;    // [2]
     uint64_t* p_full = bars + 11;
-    uint64_t* pv_done = bars + 12;   // phase j completes when the P.V of tile j has (P free, O_g readable)
+    uint64_t* pv_done = bars + 12;   // phase j completes when the P.V of tile j has (O_g readable)
     uint64_t* drain = bars + 13;
     uint64_t* sum_bar = bars + 14;   // final (max, sum) exchange between the two halves of a row
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffSlot);
@@ -159,7 +158,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&k_empty[i], 1);
             mbar_init(&v_empty[i], 1);
             mbar_init(&s_full[i], 1);
-            mbar_init(&s_empty[i], kSoftmaxWarps);
         }
         mbar_init(p_full, kSoftmaxWarps);
         mbar_init(pv_done, 1);
@@ -259,12 +257,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (lane == 0) {
             const uint32_t idesc_qk = umma_idesc_f16(kTile, kTile, false);
             const uint32_t idesc_pv = umma_idesc_f16(kTile, D, true);
-            const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
+            const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
             bool ok = mbar_wait(q_full, 0);
             auto issue_s = [&](int j) -> bool {
                 const int st = j & 1;
                 if (!mbar_wait(&k_full[st], (j >> 1) & 1)) return false;
-                if (!mbar_wait(&s_empty[j & 1], ((j >> 1) & 1) ^ 1)) return false;
+                // S(j) reuses the buffer of S(j-2)/P(j-2): it is issued after P.V(j-2), which the
+                // tensor core runs first, and P.V(j-2) waited for every softmax warp to finish that tile
                 tc_fence_after_sync();
                 const uint32_t d = tmem + C::kColS + (j & 1) * kTile;
                 const uint32_t kb = aK + st * C::kOpBytes;
@@ -289,11 +288,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const uint32_t vb = aV + st * C::kOpBytes;
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk) {
-                    // keys 0-63 of the tile add to O_0, keys 64-127 to O_1; tile 0 starts both
+                    // keys 0-63 of the tile add to O_0, keys 64-127 to O_1; tile 0 starts both.  P of
+                    // keys 64h .. 64h+63 is fp16 in columns 64h .. 64h+31 of the tile's S buffer.
                     const uint32_t d = tmem + C::kColO + (kk >> 2) * D;
-                    const uint32_t poff = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-                    umma_f16_ss(d, umma_desc_sw128(aP + poff, 16, 1024),
-                                umma_desc_sw128(vb + kk * 16 * 128, C::kChunkBytes, 1024), idesc_pv,
+                    const uint32_t pa = tmem + C::kColS + (j & 1) * kTile + (kk >> 2) * 64 + (kk & 3) * 8;
+                    umma_f16_ts(d, pa, umma_desc_sw128(vb + kk * 16 * 128, C::kChunkBytes, 1024), idesc_pv,
                                 j > 0 || (kk & 3) != 0);
                 }
                 umma_commit(pv_done);
@@ -322,7 +321,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const float qs = p.qscale;
         float m = -INFINITY, l = 0.f;                    // log2-domain running max and sum of this half
         bool ok = true;
-        uint8_t* prow = sP + g * C::kChunkBytes + r * 128;
         for (int j = 0; j < n_tiles && ok; ++j) {
             if (!(ok = mbar_wait(&s_full[j & 1], (j >> 1) & 1))) break;
             tc_fence_after_sync();
@@ -338,10 +336,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
                 for (int i = 0; i < 32; ++i) { sv[i] = __uint_as_float(r0[i]); sv[32 + i] = __uint_as_float(r1[i]); }
             }
-            // S is in registers: the buffer can take the tile after next
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_empty[j & 1]);
             if (diag) {
 #pragma unroll
                 for (int i = 0; i < 64; ++i)
@@ -372,9 +366,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 rs4[i & 3] = add_h2_f32(rs4[i & 3], pk[i]);   // the fp16 values the P.V MMA adds
             }
             l = fmaf(l, alpha, (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
-            // the P.V of tile j-1 has read P and added to O_g before either is touched
-            if (!(ok = mbar_wait(pv_done, (j & 1) ^ 1))) break;
             if (j > 0 && __any_sync(0xffffffffu, raise)) {
+                // O_g holds the sum up to tile j-1: wait for that P.V, then rescale this warp's rows
+                if (!(ok = mbar_wait(pv_done, (j & 1) ^ 1))) break;
                 tc_fence_after_sync();
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
@@ -384,11 +378,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     for (int i = 0; i < 32; ++i) v[i] *= alpha;
                     tmem_st_32cols(o_mine + c * 32, v);
                 }
-                tmem_wait_st();
             }
-#pragma unroll
-            for (int u = 0; u < 8; ++u)                               // 8 keys = one 16-byte unit of P
-                st_shared_u4(prow + ((u ^ (r & 7)) * 16), make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]));
+            // P (fp16 pairs) over the first half of this thread's S columns, which it has already read;
+            // the P.V of tile j-2, the last reader of this buffer, completed before S(j) did
+            tmem_st_32cols_u(sa, pk);
+            tmem_wait_st();
             if (j == n_tiles - 1 && kv_len < key0 + kTile) {
                 // rows of V past the sequence end may hold anything: zero them before P.V reads them
                 if (!(ok = mbar_wait(&v_full[j & 1], (j >> 1) & 1))) break;
@@ -400,9 +394,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         for (int u = 0; u < 8 / 2; ++u)
                             st_shared_u4(vrow + c * C::kChunkBytes + (g * 4 + u) * 16, make_uint4(0, 0, 0, 0));
                 }
+                fence_proxy_async_smem();                     // the zeros reach the tensor core's view
             }
             tc_fence_before_sync();
-            fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(p_full);
             if (info[2]) ok = false;
