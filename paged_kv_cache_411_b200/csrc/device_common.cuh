@@ -257,6 +257,12 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr, uint32_t
 }
 
 // Instruction descriptor for kind::f16: fp16 A and B, fp32 D, M x N, A K-major, B K- or MN-major.
+// The descriptor of the operand `bytes` further on: the start address sits in bits 0-13 in 16-byte
+// units and shared-memory addresses stay below 256 KB, so the sum never carries out of the field.
+__device__ __forceinline__ uint64_t umma_desc_advance(uint64_t desc, uint32_t bytes) {
+    return desc + (bytes >> 4);
+}
+
 __host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N, bool b_mn_major) {
     return (1u << 4) | (b_mn_major ? (1u << 16) : 0u) | (static_cast<uint32_t>(N >> 3) << 17) |
            (static_cast<uint32_t>(M >> 4) << 24);

@@ -257,7 +257,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (lane == 0) {
             const uint32_t idesc_qk = umma_idesc_f16(kTile, kTile, false);
             const uint32_t idesc_pv = umma_idesc_f16(kTile, D, true);
-            const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+            // base descriptors, built once: a k-step's operand is the base advanced by a constant
+            const uint64_t dQ = umma_desc_sw128(smem_u32(sQ), 16, 1024);
+            const uint64_t dK = umma_desc_sw128(smem_u32(sK), 16, 1024);
+            const uint64_t dV = umma_desc_sw128(smem_u32(sV), C::kChunkBytes, 1024);
             bool ok = mbar_wait(q_full, 0);
             auto issue_s = [&](int j) -> bool {
                 const int st = j & 1;
@@ -266,12 +269,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 // tensor core runs first, and P.V(j-2) waited for every softmax warp to finish that tile
                 tc_fence_after_sync();
                 const uint32_t d = tmem + C::kColS + (j & 1) * kTile;
-                const uint32_t kb = aK + st * C::kOpBytes;
+                const uint64_t dKs = umma_desc_advance(dK, st * C::kOpBytes);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-                    umma_f16_ss(d, umma_desc_sw128(aQ + off, 16, 1024), umma_desc_sw128(kb + off, 16, 1024), idesc_qk,
-                                kk > 0);
+                    umma_f16_ss(d, umma_desc_advance(dQ, off), umma_desc_advance(dKs, off), idesc_qk, kk > 0);
                 }
                 umma_commit(&s_full[j & 1]);
                 umma_commit(&k_empty[st]);
@@ -285,15 +287,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (!(ok = mbar_wait(&v_full[st], (j >> 1) & 1))) break;
                 if (info[2]) { ok = false; break; }
                 tc_fence_after_sync();
-                const uint32_t vb = aV + st * C::kOpBytes;
+                const uint64_t dVs = umma_desc_advance(dV, st * C::kOpBytes);
+                const uint32_t pbase = tmem + C::kColS + (j & 1) * kTile;
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk) {
                     // keys 0-63 of the tile add to O_0, keys 64-127 to O_1; tile 0 starts both.  P of
                     // keys 64h .. 64h+63 is fp16 in columns 64h .. 64h+31 of the tile's S buffer.
                     const uint32_t d = tmem + C::kColO + (kk >> 2) * D;
-                    const uint32_t pa = tmem + C::kColS + (j & 1) * kTile + (kk >> 2) * 64 + (kk & 3) * 8;
-                    umma_f16_ts(d, pa, umma_desc_sw128(vb + kk * 16 * 128, C::kChunkBytes, 1024), idesc_pv,
-                                j > 0 || (kk & 3) != 0);
+                    const uint32_t pa = pbase + (kk >> 2) * 64 + (kk & 3) * 8;
+                    umma_f16_ts(d, pa, umma_desc_advance(dVs, kk * 16 * 128), idesc_pv, j > 0 || (kk & 3) != 0);
                 }
                 umma_commit(pv_done);
                 umma_commit(&v_empty[st]);
