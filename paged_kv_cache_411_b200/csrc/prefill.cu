@@ -81,7 +81,7 @@ struct PCfg {
     static constexpr size_t kOffK = kOffQ + kOpBytes;
     static constexpr size_t kOffV = kOffK + size_t(kStages) * kOpBytes;
     static constexpr size_t kOffBar = kOffV + size_t(kStages) * kOpBytes;
-    static constexpr int kNumBars = 17;
+    static constexpr int kNumBars = 12;
     static constexpr size_t kOffSlot = kOffBar + kNumBars * 8;
     static constexpr size_t kOffRed = kOffSlot + 64;                 // final exchange: maxes [2][128], sums [2][128]
     // Every CTA takes all 512 TMEM columns, so the request is kept above half the SM's shared
@@ -113,13 +113,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint64_t* q_full = bars + 0;
     uint64_t* k_full = bars + 1;     // [2]
     uint64_t* v_full = bars + 3;     // [2]
-    uint64_t* k_empty = bars + 5;    // [2] released by the S MMA
-    uint64_t* v_empty = bars + 15;   // [2] released by the P.V MMA
-    uint64_t* s_full = bars + 7;     // [2]
-    uint64_t* p_full = bars + 11;
-    uint64_t* pv_done = bars + 12;   // phase j completes when the P.V of tile j has (O_g readable)
-    uint64_t* drain = bars + 13;
-    uint64_t* sum_bar = bars + 14;   // final (max, sum) exchange between the two halves of a row
+    uint64_t* s_full = bars + 5;     // [2] S(j) is in TMEM, which also frees K stage j % 2
+    uint64_t* p_full = bars + 7;
+    uint64_t* pv_done = bars + 8;    // [2] P.V(j) has landed in O_0/O_1, which also frees V stage j % 2
+    uint64_t* drain = bars + 10;
+    uint64_t* sum_bar = bars + 11;   // final (max, sum) exchange between the two halves of a row
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffSlot);
     volatile int* info = reinterpret_cast<volatile int*>(smem + C::kOffSlot + 16);   // b, qt, abort
 
@@ -155,12 +153,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int i = 0; i < 2; ++i) {
             mbar_init(&k_full[i], kIssueWarps);
             mbar_init(&v_full[i], kIssueWarps);
-            mbar_init(&k_empty[i], 1);
-            mbar_init(&v_empty[i], 1);
             mbar_init(&s_full[i], 1);
+            mbar_init(&pv_done[i], 1);
         }
         mbar_init(p_full, kSoftmaxWarps);
-        mbar_init(pv_done, 1);
         mbar_init(drain, 1);
         mbar_init(sum_bar, kSoftmaxWarps);
         mbar_init_fence();
@@ -202,7 +198,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int wsub = warp - (is_k ? kFirstKWarp : kFirstVWarp);
         const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
         uint64_t* full = is_k ? k_full : v_full;
-        uint64_t* empty = is_k ? k_empty : v_empty;
+        uint64_t* empty = is_k ? s_full : pv_done;      // stage j % 2 is free once S / P.V of tile j-2 is done
         uint8_t* base = is_k ? sK : sV;
         const uint64_t pol = l2_policy_evict_last();     // K/V tiles are re-read by the head's other q-tiles
         if (lane == 0) {
@@ -262,9 +258,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const uint64_t dK = umma_desc_sw128(smem_u32(sK), 16, 1024);
             const uint64_t dV = umma_desc_sw128(smem_u32(sV), C::kChunkBytes, 1024);
             bool ok = mbar_wait(q_full, 0);
-            auto issue_s = [&](int j) -> bool {
+            // An mbarrier answers after ~150 cycles even when its phase is complete, so this thread asks
+            // early (mbar_test_wait) and collects the answers after the MMAs it issues meanwhile; it only
+            // blocks when a phase really is still open.
+            auto issue_s = [&](int j, bool k_ready) -> bool {
                 const int st = j & 1;
-                if (!mbar_wait(&k_full[st], (j >> 1) & 1)) return false;
+                if (!k_ready && !mbar_wait(&k_full[st], (j >> 1) & 1)) return false;
                 // S(j) reuses the buffer of S(j-2)/P(j-2): it is issued after P.V(j-2), which the
                 // tensor core runs first, and P.V(j-2) waited for every softmax warp to finish that tile
                 tc_fence_after_sync();
@@ -275,17 +274,20 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
                     umma_f16_ss(d, umma_desc_advance(dQ, off), umma_desc_advance(dKs, off), idesc_qk, kk > 0);
                 }
-                umma_commit(&s_full[j & 1]);
-                umma_commit(&k_empty[st]);
+                umma_commit(&s_full[st]);
                 return true;
             };
-            if (ok) ok = issue_s(0);
+            if (ok) ok = issue_s(0, false);
+            bool k_ready = ok && n_tiles > 1 && mbar_test_wait(&k_full[1], 0);
             for (int j = 0; ok && j < n_tiles; ++j) {
-                if (j + 1 < n_tiles && !(ok = issue_s(j + 1))) break;
                 const int st = j & 1;
-                if (!(ok = mbar_wait(p_full, j & 1))) break;
-                if (!(ok = mbar_wait(&v_full[st], (j >> 1) & 1))) break;
+                const bool p_ready = mbar_test_wait(p_full, j & 1);
+                const bool v_ready = mbar_test_wait(&v_full[st], (j >> 1) & 1);
+                if (j + 1 < n_tiles && !(ok = issue_s(j + 1, k_ready))) break;
+                if (!p_ready && !(ok = mbar_wait(p_full, j & 1))) break;
+                if (!v_ready && !(ok = mbar_wait(&v_full[st], (j >> 1) & 1))) break;
                 if (info[2]) { ok = false; break; }
+                k_ready = j + 2 < n_tiles && mbar_test_wait(&k_full[st], ((j + 2) >> 1) & 1);   // for S(j+2)
                 tc_fence_after_sync();
                 const uint64_t dVs = umma_desc_advance(dV, st * C::kOpBytes);
                 const uint32_t pbase = tmem + C::kColS + (j & 1) * kTile;
@@ -297,8 +299,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     const uint32_t pa = pbase + (kk >> 2) * 64 + (kk & 3) * 8;
                     umma_f16_ts(d, pa, umma_desc_advance(dVs, kk * 16 * 128), idesc_pv, j > 0 || (kk & 3) != 0);
                 }
-                umma_commit(pv_done);
-                umma_commit(&v_empty[st]);
+                umma_commit(&pv_done[st]);
             }
             if (!ok) {
                 abort_now();
@@ -370,7 +371,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             l = fmaf(l, alpha, (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
             if (j > 0 && __any_sync(0xffffffffu, raise)) {
                 // O_g holds the sum up to tile j-1: wait for that P.V, then rescale this warp's rows
-                if (!(ok = mbar_wait(pv_done, (j & 1) ^ 1))) break;
+                if (!(ok = mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1))) break;
                 tc_fence_after_sync();
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
@@ -410,7 +411,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         __syncwarp();
         if (lane == 0) mbar_arrive(sum_bar);
         if (ok) ok = mbar_wait(sum_bar, 0);
-        if (ok) ok = mbar_wait(pv_done, (n_tiles - 1) & 1);        // the last P.V has landed in O_0, O_1
+        if (ok) ok = mbar_wait(&pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1);   // the last P.V has landed
         if (ok) {
             tc_fence_after_sync();
             const float m0 = red[r], m1 = red[128 + r];
