@@ -182,6 +182,23 @@ def _oracle_case(w, budget_tokens):
     return sample, args, tokens
 
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of the current
+# kernels on each workload at its default block size; the decode entry sums the plan, streaming and combine
+# launches of one call.  Workloads without a capture report None, and so must any entry whose kernel has
+# changed since it was taken.
+NCU_TRAFFIC_BYTES = {
+    "b256": {"decode": 2_811_811_000},
+    "b32": {"decode": 276_692_000},
+    "mixed": {"decode": 1_104_481_000, "prefill": 37_940_000},
+}
+
+
+def ncu_traffic(w, args, kernel):
+    if args.block_size:
+        return None
+    return NCU_TRAFFIC_BYTES.get(args.workload, {}).get(kernel)
+
+
 def time_oracle(w, steps, warmup, budget_tokens, min_seconds=0.0, max_steps=None):
     """Times the CPU oracle's decode on a bounded sample of the workload's sequences.
 
@@ -368,7 +385,7 @@ def run_ours(args):
             "decode_tokens_per_s_32_layers": round(S * world / (32 * ms_per_step / 1e3), 1),
             "roofline": {"kernel": "paged_attention_decode (plan + streaming kernel + combine)", "bound": "hbm",
                          "achieved": round(dec_gbs, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": round(dec_gbs / peak, 4), "traffic": None,
+                         "frac": round(dec_gbs / peak, 4), "traffic": ncu_traffic(w, args, "decode"),
                          "algorithmic_bytes_per_launch": dec_b, "avg_launch_ms": round(dec_avg_ms, 5)},
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(1e3 * e2e_max / args.steps, 4)},
@@ -382,7 +399,7 @@ def run_ours(args):
             line["roofline_prefill"] = {
                 "kernel": "paged_attention_prefill_chunk (tcgen05)", "bound": "tensor", "achieved": round(tf, 2),
                 "peak": peak_tf, "peak_kind": peak_kind + " bf16 burst (fp16 has the same nominal rate)",
-                "unit": "TFLOP/s", "frac": round(tf / peak_tf, 4), "traffic": None,
+                "unit": "TFLOP/s", "frac": round(tf / peak_tf, 4), "traffic": ncu_traffic(w, args, "prefill"),
                 "algorithmic_flops_per_launch": prefill_flops(w), "avg_launch_ms": round(pre_avg, 5)}
         if world == 1 and not args.no_cpu_baseline:
             gbs, dt, desc, threads = time_oracle(w, 1, 1, args.oracle_tokens, min_seconds=10.0, max_steps=30)
