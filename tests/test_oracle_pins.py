@@ -444,7 +444,7 @@ def test_shared_prefix_workload_refcounts():
         k = np.concatenate([kp, kx, small.k_new()[s][None]])
         v = np.concatenate([vp, vx, small.v_new()[s][None]])
         np.testing.assert_allclose(dec[s], _sdpa(small.q()[s][None], k, v, small.scale)[0], atol=1e-12)
-    # the full-size recipe's demand is the survey's closed form
+    # the full-size recipe's demand in closed form: 32 shared prefix blocks + 8 x 992 private ones
     assert owl.demand_blocks(w) == 32 + 8 * 992
     assert owl.pool_blocks(w) == math.ceil(1.1 * (32 + 8 * 992))
 
