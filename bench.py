@@ -254,7 +254,7 @@ def run_reference(args):
     per_step = oracle_tokens_for(w, args.steps + args.warmup, 120.0)
     gbs, dt, desc, threads = time_oracle(w, args.steps, args.warmup, per_step)
     line = {
-        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": 0,
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "num_seqs": w.num_seqs, "num_heads": w.num_heads, "head_dim": w.head_dim,
