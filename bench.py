@@ -492,6 +492,26 @@ def run_serve(args):
     out_p = torch.empty((max_tokens, H, D), dtype=torch.float16, device=dev)
     scale = 1 / np.sqrt(D)
     stream = torch.cuda.current_stream(dev)
+    # per-step inputs go up through one pinned staging buffer allocated once at its largest size and sent
+    # with one copy per step (an engine reuses it; pinning memory every step would cost more than the
+    # scheduling itself)
+    layout = [("slots", torch.int64, (rows,)), ("pt", torch.int32, (max_seqs, mb)), ("qs", torch.int32, (max_seqs + 1,)),
+              ("ctx", torch.int32, (max_seqs,)), ("dt", torch.int32, (max_seqs, mb)), ("dl", torch.int32, (max_seqs,))]
+    offs, total = {}, 0
+    for name, dtype, shape in layout:
+        nbytes = int(np.prod(shape)) * torch.tensor([], dtype=dtype).element_size()
+        total = (total + 255) // 256 * 256
+        offs[name] = (total, nbytes, dtype, shape)
+        total += nbytes
+    host_buf = torch.empty(total, dtype=torch.uint8).pin_memory()
+    dev_buf = torch.empty(total, dtype=torch.uint8, device=dev)
+    host_v = {k: host_buf[o:o + nb].view(dt).view(sh).numpy() for k, (o, nb, dt, sh) in offs.items()}
+    dev_v = {k: dev_buf[o:o + nb].view(dt).view(sh) for k, (o, nb, dt, sh) in offs.items()}
+
+    def stage(key, arr):
+        host_v[key][:arr.shape[0]] = arr
+        return dev_v[key][:arr.shape[0]]
+
     ends, gpu_ms, host_s = [], [], 0.0
     t_start = time.perf_counter()
     while sched.stats()["finished"] < n:
@@ -500,17 +520,18 @@ def run_serve(args):
         P, S, T = plan["num_prefill"], plan["num_decode"], plan["num_tokens"]
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if T:
-            slots = torch.from_numpy(plan["slot_mapping"]).pin_memory().to(dev, non_blocking=True)
+            slots = stage("slots", plan["slot_mapping"])
             if P:
                 _, pt, _ = alloc.pack(plan["prefill_reqs"], mb)
                 q_start = np.concatenate([[0], np.cumsum(plan["prefill_len"])]).astype(np.int32)
-                pt_d = torch.from_numpy(pt).pin_memory().to(dev, non_blocking=True)
-                qs_d = torch.from_numpy(q_start).pin_memory().to(dev, non_blocking=True)
-                ctx_d = torch.from_numpy(plan["prefill_ctx"]).pin_memory().to(dev, non_blocking=True)
+                pt_d = stage("pt", pt)
+                qs_d = stage("qs", q_start)
+                ctx_d = stage("ctx", plan["prefill_ctx"])
             if S:
                 _, dt, dl = alloc.pack(plan["decode_reqs"], mb)
-                dt_d = torch.from_numpy(dt).pin_memory().to(dev, non_blocking=True)
-                dl_d = torch.from_numpy(dl).pin_memory().to(dev, non_blocking=True)
+                dt_d = stage("dt", dt)
+                dl_d = stage("dl", dl)
+            dev_buf.copy_(host_buf, non_blocking=True)       # the step's inputs, one copy
             host_s += time.perf_counter() - h0
             ev0.record(stream)
             pk.reshape_and_cache(kpool[:T], vpool[:T], kc, vc, slots, stream=stream)
