@@ -164,6 +164,12 @@ class Scheduler:
         cfg = SchedConfig(self.max_num_seqs, self.max_num_tokens, int(bool(chunked_prefill)), int(watermark_blocks))
         self._h = c_void_p()
         check(lib().pa_sched_create(alloc._h, byref(cfg), byref(self._h)))
+        # output buffers of pa_sched_step and their ctypes pointers, made once (a step copies out its slices)
+        n, t = self.max_num_seqs, self.max_num_tokens + self.max_num_seqs
+        self._bufs = (np.empty(n, np.int64), np.empty(n, np.int32), np.empty(n, np.int32),
+                      np.empty(n, np.int64), np.empty(n, np.int32), np.empty(t, np.int64))
+        conv = (_i64p, _i32p, _i32p, _i64p, _i32p, _i64p)
+        self._ptrs = tuple(f(b) for f, b in zip(conv, self._bufs))
 
     def close(self):
         if self._h:
@@ -182,12 +188,9 @@ class Scheduler:
     def step(self) -> dict:
         """Schedule one step; returns info plus the prefill/decode entries and the slot mapping."""
         from ._lib import StepInfo
-        n, t = self.max_num_seqs, self.max_num_tokens + self.max_num_seqs
-        pr, pc, pl = np.empty(n, np.int64), np.empty(n, np.int32), np.empty(n, np.int32)
-        dr, dl, sm = np.empty(n, np.int64), np.empty(n, np.int32), np.empty(t, np.int64)
+        pr, pc, pl, dr, dl, sm = self._bufs
         info = StepInfo()
-        check(lib().pa_sched_step(self._h, byref(info), _i64p(pr), _i32p(pc), _i32p(pl), _i64p(dr), _i32p(dl),
-                                  _i64p(sm)))
+        check(lib().pa_sched_step(self._h, byref(info), *self._ptrs))
         d = info.as_dict()
         P, D, T = info.num_prefill, info.num_decode, info.num_tokens
         d.update(prefill_reqs=pr[:P].copy(), prefill_ctx=pc[:P].copy(), prefill_len=pl[:P].copy(),
