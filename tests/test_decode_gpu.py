@@ -267,3 +267,42 @@ def test_decode_over_prefix_cached_blocks(cuda_ready):
         assert np.abs(got[i] - ref).max() <= TOL
     assert tables[0][:4].tolist() == tables[1][:4].tolist()      # B and C share the 4 prompt blocks
     assert alloc.cache_stats()["hit_blocks"] == 8
+
+
+@pytest.mark.parametrize("qmul", [8.0, 16.0])
+def test_decode_sharp_softmax(cuda_ready, qmul):
+    """Scaled-up queries make a few keys dominate each row: the split-K partitions then carry very
+    different maxima and the combine's rescaling decides the result."""
+    rng = np.random.default_rng(41)
+    H, D, bs = 4, 128, 16
+    lens = [1, 15, 16, 17, 300, 777, 1500, 2047]
+    need = [-(-n // bs) for n in lens]
+    N = sum(need) + 7
+    order = rng.permutation(N)
+    kc = np.full((N, bs, H, D), np.nan, np.float16)
+    vc = np.full((N, bs, H, D), np.nan, np.float16)
+    maxb = max(need) + 1
+    tables = rng.integers(0, N, size=(len(lens), maxb)).astype(np.int32)      # wrong-but-valid padding
+    nxt = 0
+    for s, n in enumerate(lens):
+        t = order[nxt:nxt + need[s]]
+        nxt += need[s]
+        tables[s, :len(t)] = t
+        k = rng.standard_normal((n, H, D)).astype(np.float16)
+        v = rng.standard_normal((n, H, D)).astype(np.float16)
+        for j in range(n):
+            kc[t[j // bs], j % bs] = k[j]
+            vc[t[j // bs], j % bs] = v[j]
+    q = (rng.standard_normal((len(lens), H, D)) * qmul).astype(np.float16)
+    seq_lens = np.asarray(lens, np.int32)
+    scale = 1 / np.sqrt(D)
+    d = {k_: torch.from_numpy(v_).cuda() for k_, v_ in dict(q=q, kc=kc, vc=vc, t=tables, l=seq_lens).items()}
+    ws = torch.empty(pk.decode_workspace_bytes(len(lens), H, D, maxb, bs), dtype=torch.uint8, device="cuda")
+    out = torch.full_like(d["q"], float("nan"))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pk.paged_attention_decode(out, d["q"], d["kc"], d["vc"], d["t"], d["l"], scale, ws, err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    ref = oatt.paged_attention_decode(q, kc, vc, tables, seq_lens, bs, scale)
+    diff = np.abs(out.float().cpu().numpy() - ref)
+    assert diff.max() <= TOL, f"max abs error {diff.max():.3g}"

@@ -167,3 +167,20 @@ def test_prefill_sharp_softmax(cuda_ready, qmul):
     ref = oracle_prefill(case, bs, scale)
     diff = np.abs(out - ref)
     assert diff.max() <= TOL, f"max abs error {diff.max():.3g}"
+
+
+def test_prefill_many_requests(cuda_ready):
+    """Sixteen requests of random cached lengths and chunk sizes in one launch: every CTA finds its
+    (request, q-tile) among uneven neighbours."""
+    rng = np.random.default_rng(53)
+    reqs = [(int(rng.integers(0, 700)), int(rng.integers(1, 300))) for _ in range(16)]
+    case = make_case(54, 4, 128, 16, reqs)
+    scale = 1 / np.sqrt(128)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = run_prefill(case, scale, err).float().cpu().numpy()
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    ref = oracle_prefill(case, 16, scale)
+    assert np.isfinite(out).all()
+    diff = np.abs(out - ref)
+    assert diff.max() <= TOL, f"max abs error {diff.max():.3g}"
