@@ -113,3 +113,20 @@ def test_scheduler_errors():
         s.complete()
     with pytest.raises(pk.PagedKVError):
         pk.Scheduler(a, max_num_seqs=0, max_num_tokens=32)
+
+
+def test_step_results_are_the_callers_own():
+    """The binding reuses its output buffers between steps; what a step returns must not change when
+    the next step runs or when the caller writes into it."""
+    alloc = pk.BlockAllocator(64, 16)
+    sched = pk.Scheduler(alloc, max_num_seqs=4, max_num_tokens=64)
+    sched.add_request(1, 40, 3)
+    sched.add_request(2, 10, 2)
+    first = sched.step()
+    kept = {k: v.copy() for k, v in first.items() if isinstance(v, np.ndarray)}
+    sched.complete()
+    second = sched.step()
+    for k, v in kept.items():
+        assert np.array_equal(first[k], v), k
+    first["slot_mapping"][:] = -7
+    assert not np.any(second["slot_mapping"] == -7)
