@@ -522,15 +522,14 @@ def run_serve(args):
         if T:
             slots = stage("slots", plan["slot_mapping"])
             if P:
-                _, pt, _ = alloc.pack(plan["prefill_reqs"], mb)
+                alloc.pack(plan["prefill_reqs"], mb, tables=host_v["pt"][:P])     # straight into staging
                 q_start = np.concatenate([[0], np.cumsum(plan["prefill_len"])]).astype(np.int32)
-                pt_d = stage("pt", pt)
+                pt_d = dev_v["pt"][:P]
                 qs_d = stage("qs", q_start)
                 ctx_d = stage("ctx", plan["prefill_ctx"])
             if S:
-                _, dt, dl = alloc.pack(plan["decode_reqs"], mb)
-                dt_d = stage("dt", dt)
-                dl_d = stage("dl", dl)
+                alloc.pack(plan["decode_reqs"], mb, tables=host_v["dt"][:S], lens=host_v["dl"][:S])
+                dt_d, dl_d = dev_v["dt"][:S], dev_v["dl"][:S]
             dev_buf.copy_(host_buf, non_blocking=True)       # the step's inputs, one copy
             host_s += time.perf_counter() - h0
             ev0.record(stream)

@@ -102,11 +102,19 @@ class BlockAllocator:
         st = lib().pa_alloc_slots(self._h, req, pos_begin, n, _i64p(out))
         return st, out
 
-    def pack(self, reqs, max_blocks: int):
+    def pack(self, reqs, max_blocks: int, tables=None, lens=None):
+        """Block tables [n, max_blocks] (padding -1) and lengths [n] of the requests; written into the given
+        C-contiguous int32 arrays when passed (e.g. views of a pinned staging buffer), else into new ones."""
         r = np.ascontiguousarray(reqs, dtype=np.int64)
-        tables = np.empty((len(r), max_blocks), dtype=np.int32)
-        lens = np.empty(len(r), dtype=np.int32)
-        st = lib().pa_alloc_pack(self._h, _i64p(r), len(r), max_blocks, _i32p(tables), _i32p(lens))
+        n = len(r)
+        if tables is None:
+            tables = np.empty((n, max_blocks), dtype=np.int32)
+        if lens is None:
+            lens = np.empty(n, dtype=np.int32)
+        if (tables.dtype != np.int32 or tables.shape != (n, max_blocks) or not tables.flags.c_contiguous
+                or lens.dtype != np.int32 or lens.shape != (n,) or not lens.flags.c_contiguous):
+            raise ValueError("pack: tables must be int32 [n, max_blocks] and lens int32 [n], C-contiguous")
+        st = lib().pa_alloc_pack(self._h, _i64p(r), n, max_blocks, _i32p(tables), _i32p(lens))
         return st, tables, lens
 
     def stats(self) -> dict:
