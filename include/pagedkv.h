@@ -359,6 +359,8 @@ size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_heads, int32_t he
  * max_blocks, block_size) bytes, 256-byte aligned, caller-owned scratch whose
  * contents need no initialisation and are clobbered; two launches in flight
  * at once must not share it.
+ * scale: the softmax temperature (1/sqrt(head_dim) for standard attention);
+ * it must be finite and > 0, anything else returns INVALID_ARG.
  * The work is split flash-decoding style into partitions of the sequence
  * combined with the exact log-sum-exp rule, so the result does not depend on
  * the physical placement of the blocks (bitwise) and matches a float64
@@ -383,7 +385,10 @@ pa_status pa_paged_attention_decode(pa_half* out, const pa_half* q,
  * until the process exits.  A batch whose pa_decode_workspace_bytes exceeds
  * that returns PA_ERR_INVALID_ARG with a message saying so.  The first call on
  * a device looks the array's address up (cudaGetSymbolAddress, with that
- * device current); make that first call before any stream capture.  Calls on
+ * device current); make that first call before any stream capture.  The
+ * address is kept for the life of the process: after cudaDeviceReset (which
+ * destroys the device's copy of the array) it is stale, so a process that
+ * resets a device must not call this entry point on it again.  Calls on
  * one device share the array: calls whose kernels may overlap on the GPU race
  * and must be serialised by the caller.  Allocates nothing.
  * Errors: as pa_paged_attention_decode. */
@@ -405,6 +410,7 @@ pa_status pa_paged_attention_decode_noalloc(pa_half* out, const pa_half* q,
  * first).  q, out: device fp16 [num_tokens][num_heads][head_dim];
  * block_tables: device int32 [num_reqs][max_blocks]; ctx_before: device int32
  * [num_reqs].  Rows of out not covered by any request are left unwritten.
+ * scale must be finite and > 0 (INVALID_ARG otherwise).
  * QK^T and PV run on the tcgen05 tensor cores (fp16 operands, fp32 TMEM
  * accumulators); the softmax runs in fp32.
  * Errors: INVALID_ARG, UNSUPPORTED, CUDA. */

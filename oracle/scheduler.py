@@ -74,8 +74,21 @@ class Scheduler:
                    if self._decoding(self.reqs[r]) and self.bm.seq_lens[r] % bs == 0)
 
     def step(self):
-        bs = self.bm.block_size
         info = dict(step=self.steps, num_admitted=0, num_preempted=0, num_finished=0)
+        self._free_finished(info)
+        need = self._preempt(info)
+        self._admit(info, need)
+        self.last_prefill, self.last_decode = [], []
+        dec_slots = self._schedule_decodes()
+        pre_slots = self._schedule_prefills(self.max_num_tokens)
+        info.update(num_prefill=len(self.last_prefill), num_decode=len(self.last_decode),
+                    num_tokens=len(pre_slots) + len(dec_slots),
+                    prefill=list(self.last_prefill), decode=list(self.last_decode),
+                    slot_mapping=pre_slots + dec_slots)
+        return info
+
+    # §2.2 step 1: requests that emitted their last token give their blocks back
+    def _free_finished(self, info):
         keep = []
         for r in self.running:
             if self.reqs[r].state == FINISHED:
@@ -84,6 +97,9 @@ class Scheduler:
             else:
                 keep.append(r)
         self.running = keep
+
+    # §5.4 strategy 1: preempt the newest running request while the decodes lack blocks
+    def _preempt(self, info):
         need = self._need()
         while need > self.bm._available() and self.running:
             v = self.running.pop()
@@ -96,6 +112,11 @@ class Scheduler:
             self.waiting.appendleft(v)
             info["num_preempted"] += 1
             need = self._need()
+        return need
+
+    # §2.2 step 2 with §5.3's watermark: admit in arrival order while seats and blocks last
+    def _admit(self, info, need):
+        bs = self.bm.block_size
         while len(self.running) < self.max_num_seqs and self.waiting:
             r = self.waiting[0]
             q = self.reqs[r]
@@ -107,16 +128,22 @@ class Scheduler:
             q.prefilled = 0
             self.running.append(r)
             info["num_admitted"] += 1
-        self.last_prefill, self.last_decode = [], []
-        dec_slots, pre_slots = [], []
+
+    # §2.2 step 3, decode half: one token for every fully prefilled request
+    def _schedule_decodes(self):
+        slots = []
         for r in self.running:
             if not self._decoding(self.reqs[r]):
                 continue
             st, slot = self.bm.append_token(r)
             assert st == OK
-            dec_slots.append(slot)
+            slots.append(slot)
             self.last_decode.append((r, self.bm.seq_lens[r]))
-        budget = self.max_num_tokens
+        return slots
+
+    # §2.2 step 3, prefill half, with §4.3's chunks: prefill tokens share the step's budget
+    def _schedule_prefills(self, budget):
+        slots = []
         for r in self.running:
             q = self.reqs[r]
             if q.state != RUNNING or q.prefilled >= q.to_prefill:
@@ -125,17 +152,13 @@ class Scheduler:
             chunk = min(remaining, budget) if self.chunked else (remaining if remaining <= budget else 0)
             if chunk <= 0:
                 continue
-            st, slots = self.bm.append_tokens(r, chunk)
+            st, s = self.bm.append_tokens(r, chunk)
             if st == OOM:
                 continue
-            pre_slots += slots
+            slots += s
             self.last_prefill.append((r, q.prefilled, chunk))
             budget -= chunk
-        info.update(num_prefill=len(self.last_prefill), num_decode=len(self.last_decode),
-                    num_tokens=len(pre_slots) + len(dec_slots),
-                    prefill=list(self.last_prefill), decode=list(self.last_decode),
-                    slot_mapping=pre_slots + dec_slots)
-        return info
+        return slots
 
     def complete(self):
         now = self.steps

@@ -197,7 +197,7 @@ def build(w: si.Workload, seqs=None) -> OracleStep:
     if w.shared_prefix:
         _check(bm.free(si.PREFIX_REQ))
 
-    max_blocks = max(blocks_needed(n, bs) for n in w.decode_lens)
+    max_blocks = max((blocks_needed(n, bs) for n in w.decode_lens), default=1)
     st, tables, lens = bm.pack(list(range(w.num_seqs)), max_blocks)
     _check(st)
     return OracleStep(

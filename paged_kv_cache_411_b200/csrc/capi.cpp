@@ -89,7 +89,8 @@ pa_status pa_paged_attention_decode(pa_half* out, const pa_half* q, const pa_hal
                     num_heads, head_dim, block_size);
     if (static_cast<int64_t>(max_blocks) * block_size > (1 << 30))
         return fail(PA_ERR_INVALID_ARG, "pa_paged_attention_decode: max_blocks*block_size too large");
-    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "pa_paged_attention_decode: scale is not finite");
+    if (!std::isfinite(scale) || !(scale > 0.f))
+        return fail(PA_ERR_INVALID_ARG, "pa_paged_attention_decode: scale must be finite and > 0");
     if (num_seqs == 0) return PA_OK;
     if (num_blocks == 0 || max_blocks == 0)
         return fail(PA_ERR_INVALID_ARG, "pa_paged_attention_decode: empty pool or table with sequences to decode");
@@ -124,7 +125,8 @@ pa_status pa_paged_attention_prefill_chunk(pa_half* out, const pa_half* q, const
     if (!pagedkv::prefill_supported(num_heads, head_dim, block_size))
         return fail(PA_ERR_UNSUPPORTED, "pa_paged_attention_prefill_chunk: no kernel for num_heads=%d head_dim=%d block_size=%d",
                     num_heads, head_dim, block_size);
-    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "pa_paged_attention_prefill_chunk: scale is not finite");
+    if (!std::isfinite(scale) || !(scale > 0.f))
+        return fail(PA_ERR_INVALID_ARG, "pa_paged_attention_prefill_chunk: scale must be finite and > 0");
     if (static_cast<int64_t>(max_blocks) * block_size > (1 << 30))
         return fail(PA_ERR_INVALID_ARG, "pa_paged_attention_prefill_chunk: max_blocks*block_size too large");
     if (num_reqs == 0 || num_tokens == 0) return PA_OK;

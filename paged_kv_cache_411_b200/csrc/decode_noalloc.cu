@@ -71,6 +71,9 @@ extern "C" pa_status pa_paged_attention_decode_noalloc(pa_half* out, const pa_ha
                                                        int32_t* err_flag, void* stream) {
     if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || block_size <= 0 || max_blocks < 0)
         return pagedkv::fail(PA_ERR_INVALID_ARG, "pa_paged_attention_decode_noalloc: bad sizes");
+    // the workspace arithmetic below is only meaningful inside the decode entry point's own limit
+    if (static_cast<int64_t>(max_blocks) * block_size > (1 << 30))
+        return pagedkv::fail(PA_ERR_INVALID_ARG, "pa_paged_attention_decode_noalloc: max_blocks*block_size too large");
     const size_t need = pagedkv::decode_workspace_bytes(num_seqs, num_heads, head_dim, max_blocks, block_size);
     if (need > kNoallocScratchBytes)
         return pagedkv::fail(PA_ERR_INVALID_ARG,

@@ -209,7 +209,7 @@ def build(w: si.Workload, device="cuda", pad="neg1", max_blocks: Optional[int] =
     k_parts.append(w.k_new())
     v_parts.append(w.v_new())
 
-    need = max(_ceil_div(n, bs) for n in w.decode_lens)
+    need = max((_ceil_div(n, bs) for n in w.decode_lens), default=1)
     mb = need if max_blocks is None else max(need, max_blocks)
     st, tables, lens = r.alloc.pack(np.arange(w.num_seqs), mb)
     _ok(st)

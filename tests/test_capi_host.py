@@ -61,10 +61,46 @@ def test_device_entry_points_reject_bad_arguments_on_host():
     assert lib.pa_reshape_and_cache(None, None, None, None, None, 0, 4, 64, 16, 4, None, None) == pk.PA_OK
     assert lib.pa_paged_attention_decode(None, None, None, None, None, None, 0, 4, 64, 16, 4, 4, 0.1,
                                          None, 0, None, None) == pk.PA_OK
-    # misaligned workspace / too small workspace
     assert pk.decode_workspace_bytes(4, 4, 64, 3, 16) > 0
     assert pk.decode_workspace_bytes(-1, 4, 64, 3, 16) == 0
-    assert "decode" in pk.last_error() or True
+
+
+# Stand-in addresses: every call below fails a host-side check before anything is launched, so these
+# are never dereferenced (the checks look only at their values).
+_A = 1 << 20            # 256-byte aligned
+_BUF = [_A + i * (1 << 16) for i in range(6)]
+
+
+def _decode_call(ws, ws_bytes, scale=0.125, S=4, H=4, D=64, bs=16, mb=3, nb=16):
+    return pk.lib().pa_paged_attention_decode(*_BUF, S, H, D, bs, mb, nb, scale, ws, ws_bytes, None, None)
+
+
+def test_decode_rejects_misaligned_or_small_workspace():
+    need = pk.decode_workspace_bytes(4, 4, 64, 3, 16)
+    assert _decode_call(_A + 64, need) == pk.PA_ERR_INVALID_ARG
+    assert "256-byte aligned" in pk.last_error()
+    assert _decode_call(_A, need - 1) == pk.PA_ERR_INVALID_ARG
+    assert f"< {need}" in pk.last_error()
+    assert _decode_call(None, need) == pk.PA_ERR_INVALID_ARG
+    assert "NULL" in pk.last_error()
+    # a misaligned fp16 buffer is refused before the workspace is looked at
+    bad = list(_BUF)
+    bad[1] += 2
+    assert pk.lib().pa_paged_attention_decode(*bad, 4, 4, 64, 16, 3, 16, 0.125, _A, need, None, None) == \
+        pk.PA_ERR_INVALID_ARG
+    assert "16-byte aligned" in pk.last_error()
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.125, float("nan"), float("inf")])
+def test_attention_entry_points_refuse_bad_scale(scale):
+    """The softmax temperature must be finite and positive: decode and prefill refuse anything else
+    before launching (the prefill kernel takes its row maximum on unscaled scores)."""
+    need = pk.decode_workspace_bytes(4, 4, 64, 3, 16)
+    assert _decode_call(_A, need, scale=scale) == pk.PA_ERR_INVALID_ARG
+    assert "scale" in pk.last_error()
+    st = pk.lib().pa_paged_attention_prefill_chunk(*_BUF, _A, 1, 32, 4, 64, 16, 3, 16, scale, None, None)
+    assert st == pk.PA_ERR_INVALID_ARG
+    assert "scale" in pk.last_error()
 
 
 def test_workspace_bytes_grow_with_shape():

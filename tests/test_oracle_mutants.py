@@ -9,9 +9,14 @@ import numpy as np
 import pytest
 
 import test_oracle_pins as pins
+import test_oracle_serving_pins as spins
+import test_prefix_cache as ppins
 from oracle import attention as oatt
 from oracle import block_manager as obm
+from oracle import prefix_cache as opc
+from oracle import scheduler as osch
 from oracle import sizes
+from oracle import swap as oswap
 
 _orig_softmax = oatt.softmax_attention
 _orig_gather = oatt.gather_sequence
@@ -117,6 +122,182 @@ class _NoRefcountBM(obm.BlockManager):
         return obm.OK
 
 
+# ---- step driver ([CB-PA] §2.2, §4.3, §5.3, §5.4)
+_Sched = osch.Scheduler
+
+
+class _DecodesUseBudget(_Sched):
+    def _schedule_prefills(self, budget):
+        return super()._schedule_prefills(budget - len(self.last_decode))
+
+
+class _PrefillBeforeDecode(_Sched):
+    def step(self):
+        info = dict(step=self.steps, num_admitted=0, num_preempted=0, num_finished=0)
+        self._free_finished(info)
+        need = self._preempt(info)
+        self._admit(info, need)
+        self.last_prefill, self.last_decode = [], []
+        pre_slots = self._schedule_prefills(self.max_num_tokens)
+        dec_slots = self._schedule_decodes()
+        info.update(num_prefill=len(self.last_prefill), num_decode=len(self.last_decode),
+                    num_tokens=len(pre_slots) + len(dec_slots), prefill=list(self.last_prefill),
+                    decode=list(self.last_decode), slot_mapping=pre_slots + dec_slots)
+        return info
+
+
+class _AdmitPastMaxSeqs(_Sched):
+    def _admit(self, info, need):
+        self.max_num_seqs += 1
+        try:
+            super()._admit(info, need)
+        finally:
+            self.max_num_seqs -= 1
+
+
+class _WatermarkOffByOne(_Sched):
+    def _admit(self, info, need):
+        super()._admit(info, need + 1)
+
+
+class _WatermarkIgnoresDecodes(_Sched):
+    def _admit(self, info, need):
+        super()._admit(info, 0)
+
+
+class _PreemptOldest(_Sched):
+    def _preempt(self, info):
+        self.running.reverse()
+        try:
+            return super()._preempt(info)
+        finally:
+            self.running.reverse()
+
+
+class _PreemptedToBack(_Sched):
+    def _preempt(self, info):
+        n = len(self.waiting)
+        need = super()._preempt(info)
+        k = info["num_preempted"]
+        if k:
+            victims = [self.waiting.popleft() for _ in range(k)]
+            self.waiting.extend(reversed(victims))
+        assert len(self.waiting) == n + k
+        return need
+
+
+class _RecomputePromptOnly(_Sched):
+    def _preempt(self, info):
+        need = super()._preempt(info)
+        for r in list(self.waiting)[:info["num_preempted"]]:
+            self.reqs[r].to_prefill = self.reqs[r].prompt_len
+        return need
+
+
+# ---- swap ([CB-PA] §4.4)
+_orig_move = oswap._move
+
+
+def _free_before_allocate(src, dst, req, src_k, src_v, dst_k, dst_v):
+    if req not in src.block_tables:
+        return obm.NOT_FOUND
+    table, n = list(src.block_tables[req]), src.seq_lens[req]
+    src.free(req)
+    st = dst.allocate(req, n)
+    if st == obm.OK and src_k is not None:
+        for s_, d in zip(table, dst.block_tables[req]):
+            dst_k[d] = src_k[s_]
+            dst_v[d] = src_v[s_]
+    return st
+
+
+def _whole_blocks_length(src, dst, req, src_k, src_v, dst_k, dst_v):
+    st = _orig_move(src, dst, req, src_k, src_v, dst_k, dst_v)
+    if st == obm.OK:
+        dst.seq_lens[req] = len(dst.block_tables[req]) * dst.block_size
+    return st
+
+
+def _copies_reversed(src, dst, req, src_k, src_v, dst_k, dst_v):
+    if req not in src.block_tables:
+        return obm.NOT_FOUND
+    if req in dst.block_tables:
+        return obm.EXISTS
+    st = dst.allocate(req, src.seq_lens[req])
+    if st != obm.OK:
+        return st
+    if src_k is not None:
+        for s_, d in zip(src.block_tables[req], reversed(dst.block_tables[req])):
+            dst_k[d] = src_k[s_]
+            dst_v[d] = src_v[s_]
+    return src.free(req)
+
+
+def _k_only(src, dst, req, src_k, src_v, dst_k, dst_v):
+    if req not in src.block_tables:
+        return obm.NOT_FOUND
+    if req in dst.block_tables:
+        return obm.EXISTS
+    st = dst.allocate(req, src.seq_lens[req])
+    if st != obm.OK:
+        return st
+    if src_k is not None:
+        for s_, d in zip(src.block_tables[req], dst.block_tables[req]):
+            dst_k[d] = src_k[s_]
+    return src.free(req)
+
+
+# ---- prefix cache ([CB-PA] §4.1, §4.2)
+_PC = opc.PrefixCachingBlockManager
+
+
+class _EvictMru(_PC):
+    def _take(self):
+        if self.free_blocks:
+            return super()._take()
+        b, _ = self.lru.popitem(last=True)
+        del self.cache[self.block_node[b]]
+        self.block_node[b] = -1
+        self.evictions += 1
+        self.refcount[b] += 1
+        return b
+
+
+class _ParkInTableOrder(_PC):
+    def _release(self, table):
+        zero = []
+        for b in table:
+            self.refcount[b] -= 1
+            if self.refcount[b] == 0:
+                zero.append(b)
+        for b in zero:
+            if self.block_node[b] < 0:
+                self.free_blocks.append(b)
+            else:
+                self.lru[b] = None
+
+
+class _HashBlockAlone(_PC):
+    def _node(self, parent, block_tokens, create):
+        return super()._node(-1, block_tokens, create)
+
+
+class _RegisterPartialBlock(_PC):
+    def allocate_cached(self, req, tokens):
+        st, cached = super().allocate_cached(req, tokens)
+        n, bs = len(tokens), self.block_size
+        if st == obm.OK and n % bs:
+            parent = -1
+            for i in range(n // bs):
+                parent = self._node(parent, [int(t) for t in tokens[i * bs:(i + 1) * bs]], create=True)
+            node = self._node(parent, [int(t) for t in tokens[(n // bs) * bs:]], create=True)
+            b = self.block_tables[req][-1]
+            if node not in self.cache:
+                self.cache[node] = b
+                self.block_node[b] = node
+        return st, cached
+
+
 def _floor_blocks(n, bs):
     return n // bs
 
@@ -154,6 +335,38 @@ MUTANTS = [
      [lambda: pins.test_blocks_needed_is_smallest_cover(16)]),
     ("kv bytes drop the K+V factor", sizes, "kv_bytes_per_token", _kv_no_two,
      [lambda: pins.test_kv_bytes_per_token_matches_page()]),
+    ("scheduler counts decodes against the prefill budget", osch, "Scheduler", _DecodesUseBudget,
+     [lambda: spins.run_oracle_scheduler_trace(spins._case("timeline"))]),
+    ("scheduler gives prefills their blocks before decodes", osch, "Scheduler", _PrefillBeforeDecode,
+     [lambda: spins.run_oracle_scheduler_trace(spins._case("timeline"))]),
+    ("scheduler admits past max_num_seqs", osch, "Scheduler", _AdmitPastMaxSeqs,
+     [lambda: spins.run_oracle_scheduler_trace(spins._case("timeline"))]),
+    ("watermark needs one block more", osch, "Scheduler", _WatermarkOffByOne,
+     [lambda: spins.run_oracle_scheduler_trace(spins._case("watermark_boundary_admits"))]),
+    ("watermark ignores the decodes' blocks", osch, "Scheduler", _WatermarkIgnoresDecodes,
+     [lambda: spins.run_oracle_scheduler_trace(spins._case("watermark_counts_decode_needs"))]),
+    ("preemption takes the oldest request", osch, "Scheduler", _PreemptOldest,
+     [lambda: spins.run_oracle_scheduler_trace(spins._case("preemption"))]),
+    ("preempted request goes to the back of the queue", osch, "Scheduler", _PreemptedToBack,
+     [lambda: spins.run_oracle_scheduler_trace(spins._case("preemption"))]),
+    ("preempted request recomputes only its prompt", osch, "Scheduler", _RecomputePromptOnly,
+     [lambda: spins.run_oracle_scheduler_trace(spins._case("preemption"))]),
+    ("swap frees the source before allocating", oswap, "_move", _free_before_allocate,
+     [lambda: spins.run_oracle_swap_trace()]),
+    ("swap gives the destination whole blocks of tokens", oswap, "_move", _whole_blocks_length,
+     [lambda: spins.run_oracle_swap_trace()]),
+    ("swap copies blocks in reverse order", oswap, "_move", _copies_reversed,
+     [lambda: spins.run_oracle_swap_trace()]),
+    ("swap leaves V behind", oswap, "_move", _k_only,
+     [lambda: spins.run_oracle_swap_trace()]),
+    ("prefix cache evicts the most recent block", opc, "PrefixCachingBlockManager", _EvictMru,
+     [lambda: ppins.test_oracle_follows_hand_trace()]),
+    ("prefix cache parks blocks in table order", opc, "PrefixCachingBlockManager", _ParkInTableOrder,
+     [lambda: ppins.test_oracle_follows_hand_trace()]),
+    ("prefix cache hashes a block without its prefix", opc, "PrefixCachingBlockManager", _HashBlockAlone,
+     [lambda: ppins.test_shared_system_prompt_is_stored_once()]),
+    ("prefix cache registers the partial last block", opc, "PrefixCachingBlockManager", _RegisterPartialBlock,
+     [lambda: ppins.test_oracle_follows_hand_trace()]),
 ]
 
 

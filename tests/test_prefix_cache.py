@@ -9,6 +9,7 @@ from hypothesis import strategies as st
 import paged_kv_cache_411_b200 as pk
 from conftest import golden
 from oracle import block_manager as obm
+from oracle import prefix_cache as opc
 from oracle.prefix_cache import PrefixCachingBlockManager
 
 _NAMES = {pk.PA_OK: obm.OK, pk.PA_ERR_OOM: obm.OOM, pk.PA_ERR_NOT_FOUND: obm.NOT_FOUND,
@@ -17,7 +18,7 @@ _NAMES = {pk.PA_OK: obm.OK, pk.PA_ERR_OOM: obm.OOM, pk.PA_ERR_NOT_FOUND: obm.NOT
 
 def test_oracle_follows_hand_trace():
     g = golden("prefix_cache_trace.json")
-    bm = PrefixCachingBlockManager(g["num_blocks"], g["block_size"])
+    bm = opc.PrefixCachingBlockManager(g["num_blocks"], g["block_size"])
     for op in g["ops"]:
         kind = op[0]
         if kind == "allocate_cached":
@@ -46,7 +47,7 @@ def test_shared_system_prompt_is_stored_once():
     system = rng.integers(0, 32000, 3 * bs).tolist()
     q1 = rng.integers(0, 32000, 20).tolist()
     q2 = rng.integers(0, 32000, 25).tolist()
-    bm = PrefixCachingBlockManager(32, bs)
+    bm = opc.PrefixCachingBlockManager(32, bs)
     assert bm.allocate_cached(1, system + q1) == (obm.OK, 0)
     assert bm.allocate_cached(2, system + q2) == (obm.OK, 3 * bs)
     assert bm.block_tables[1][:3] == bm.block_tables[2][:3]
@@ -61,6 +62,8 @@ def test_shared_system_prompt_is_stored_once():
     # identical block content after a different prefix is a different block
     other = rng.integers(0, 32000, bs).tolist()
     assert bm.allocate_cached(5, other + system[bs:2 * bs]) == (obm.OK, 0)
+    # and a block seen only after a prefix is no hit at the start of a prompt
+    assert bm.allocate_cached(6, system[bs:2 * bs] + [1]) == (obm.OK, 0)
 
 
 def _replay(N, bs, log, vocab):

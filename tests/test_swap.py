@@ -59,46 +59,78 @@ def test_swap_argument_errors():
         pk.swap_blocks(None, None, None, None, [[0, 5]], 16, 4, 4)     # pair outside the pools
 
 
+def _bits(a):
+    return np.ascontiguousarray(a).view(np.int16)
+
+
 @pytest.mark.gpu
-def test_swap_round_trip_on_gpu(cuda_ready):
-    """Swap three sequences of a batch out to pinned host memory (bit-exact copies), decode the
-    others, swap them back into different GPU blocks, and decode all: identical outputs."""
+def test_swap_round_trip_matches_oracle(cuda_ready):
+    """Swap three sequences of a batch out to a pinned host pool and back into different GPU blocks,
+    moving the same requests with the oracle's SwappingManager on NumPy copies of the same starting
+    pools ([CB-PA] §4.4).  After every move the GPU pool and the host pool equal the oracle's pools
+    bit for bit (NaN-poisoned spare rows included), and the tables and free lists match; decode over
+    the moved blocks then matches oracle attention over the oracle's pool and is bitwise the decode
+    from before the round trip."""
+    from oracle import workloads as owl
     w = si.Workload(name="swap", seed=12, num_heads=8, head_dim=128, block_size=16,
                     decode_lens=(100, 37, 513, 16, 260, 1), pool_factor=2.0)
     ds = pwl.build(w)
+    o = owl.build(w)
+    bs = w.block_size
+    kc, vc = o.k_cache.copy(), o.v_cache.copy()
+    oatt.reshape_and_cache(kc, vc, o.k_step, o.v_step, o.slot_mapping, bs)
     pk.reshape_and_cache(ds.k_step, ds.v_step, ds.k_cache, ds.v_cache, ds.slot_mapping)
     S, H, D = ds.q.shape
-    bs = w.block_size
     mb = ds.max_blocks
     ws = torch.empty(pk.decode_workspace_bytes(S, H, D, mb, bs), dtype=torch.uint8, device="cuda")
     ref = torch.empty_like(ds.q)
     pk.paged_attention_decode(ref, ds.q, ds.k_cache, ds.v_cache, ds.block_tables, ds.seq_lens, w.scale, ws)
-    gpu = ds.alloc
+    torch.cuda.synchronize()
+    assert np.array_equal(_bits(ds.k_cache.cpu().numpy()), _bits(kc))
+
+    gpu, ogpu = ds.alloc, o.bm
     NC = 64
-    cpu = pk.BlockAllocator(NC, bs)
+    cpu, ocpu = pk.BlockAllocator(NC, bs), obm.BlockManager(NC, bs)
+    sm = SwappingManager(ogpu, ocpu)
     ck = torch.zeros((NC, bs, H, D), dtype=torch.float16).pin_memory()
     cv = torch.zeros_like(ck).pin_memory()
+    ock, ocv = np.zeros((NC, bs, H, D), np.float16), np.zeros((NC, bs, H, D), np.float16)
     block_bytes = bs * H * D * 2
+
+    def check_same(what):
+        torch.cuda.synchronize()
+        assert np.array_equal(_bits(ds.k_cache.cpu().numpy()), _bits(kc)), what
+        assert np.array_equal(_bits(ds.v_cache.cpu().numpy()), _bits(vc)), what
+        assert np.array_equal(_bits(ck.numpy()), _bits(ock)), what
+        assert np.array_equal(_bits(cv.numpy()), _bits(ocv)), what
+        assert gpu.free_list().tolist() == ogpu.free_blocks, what
+        assert cpu.free_list().tolist() == ocpu.free_blocks, what
+        for r in list(range(S)) + [99]:
+            assert gpu.get_block_table(r)[1].tolist() == ogpu.get_block_table(r)[1], (what, r)
+            assert cpu.get_block_table(r)[1].tolist() == ocpu.get_block_table(r)[1], (what, r)
+
     before = {r: gpu.get_block_table(r)[1] for r in (0, 2, 4)}
-    gk_host, gv_host = ds.k_cache.cpu().numpy(), ds.v_cache.cpu().numpy()
     for r in (0, 2, 4):
         assert pk.swap_out(gpu, cpu, r, ds.k_cache, ds.v_cache, ck, cv, block_bytes) == pk.PA_OK
-    torch.cuda.synchronize()
-    for r in (0, 2, 4):
-        ct = cpu.get_block_table(r)[1]
-        assert np.array_equal(ck.numpy()[ct].view(np.int16), gk_host[before[r]].view(np.int16))
-        assert np.array_equal(cv.numpy()[ct].view(np.int16), gv_host[before[r]].view(np.int16))
+        assert sm.swap_out(r, kc, vc, ock, ocv) == obm.OK
+        check_same(f"swap_out {r}")
         assert gpu.seq_len(r)[0] == pk.PA_ERR_NOT_FOUND
     # reuse the freed GPU blocks for a filler request, then swap back in: new physical blocks
     filler_tokens = sum(len(v) for v in before.values()) * bs // 2
     assert gpu.allocate(99, filler_tokens) == pk.PA_OK
+    assert ogpu.allocate(99, filler_tokens) == obm.OK
     for r in (0, 2, 4):
         assert pk.swap_in(gpu, cpu, r, ds.k_cache, ds.v_cache, ck, cv, block_bytes) == pk.PA_OK
+        assert sm.swap_in(r, kc, vc, ock, ocv) == obm.OK
+        check_same(f"swap_in {r}")
     st_, tables, lens = gpu.pack(np.arange(S), mb)
     assert st_ == pk.PA_OK
     assert any(not np.array_equal(tables[r][:len(before[r])], before[r]) for r in (0, 2, 4))
     out = torch.empty_like(ds.q)
     pk.paged_attention_decode(out, ds.q, ds.k_cache, ds.v_cache, torch.from_numpy(tables).cuda(),
                               torch.from_numpy(lens).cuda(), w.scale, ws)
+    torch.cuda.synchronize()
+    want = oatt.paged_attention_decode(o.q, kc, vc, tables, lens, bs, w.scale)
+    assert float(np.abs(out.float().cpu().numpy() - want).max()) <= 2e-3
     assert torch.equal(out, ref)
     assert cpu.stats()["num_free"] == NC
