@@ -94,6 +94,23 @@ const char* pa_status_string(pa_status s);
 /* PA_OK if `flag_value` (a read-back err_flag) is 0, else PA_ERR_DEVICE_CHECK. */
 pa_status pa_check_device_flag(int32_t flag_value);
 
+/* Kernels a failure-detection test can stall. */
+enum { PA_KERNEL_DECODE = 1, PA_KERNEL_PREFILL = 2 };
+
+/* Test hook for the device-side failure detection.  Every wait inside the
+ * attention kernels is bounded (2 s); when one runs out the kernel ORs
+ * PA_DEVCHK_TIMEOUT into err_flag, stops its other roles, lets the copies and
+ * tensor-core operations it issued complete, frees what it holds and returns,
+ * so the CUDA context stays usable.  This call makes the NEXT launch of
+ * `kernel` in this process exercise that path: its consumer role (decode:
+ * the softmax warps; prefill: the softmax warps) first waits on a barrier
+ * that nothing completes, and every pipeline wait of that launch is bounded by
+ * wait_limit_ns instead of 2 s (the final drain waits keep 2 s).  The launch
+ * then returns with PA_DEVCHK_TIMEOUT set and its output undefined; later
+ * launches are normal.  Not for production use.
+ * Errors: INVALID_ARG (unknown kernel, wait_limit_ns 0 or above 2e9). */
+pa_status pa_debug_inject_stall(int32_t kernel, uint64_t wait_limit_ns);
+
 /* ---- host block allocator ([CB-PA] §3.2 BlockManager, §4.1 shared prefix) --
  *
  * Free list: starts as init_free_order (or 0..num_blocks-1 when NULL); every

@@ -17,7 +17,7 @@ from ctypes import POINTER, byref, c_int32, c_int64, c_void_p
 import numpy as np
 
 from ._lib import (PA_DEVCHK_BLOCK_ID, PA_DEVCHK_QUERY_RANGE, PA_DEVCHK_SEQ_LEN, PA_DEVCHK_SLOT,
-                   PA_DEVCHK_TIMEOUT, PA_ERR_CUDA, PA_ERR_DEVICE_CHECK, PA_ERR_EXISTS, PA_ERR_INVALID_ARG,
+                   PA_DEVCHK_TIMEOUT, PA_KERNEL_DECODE, PA_KERNEL_PREFILL, PA_ERR_CUDA, PA_ERR_DEVICE_CHECK, PA_ERR_EXISTS, PA_ERR_INVALID_ARG,
                    PA_ERR_NOT_FOUND, PA_ERR_OOM, PA_ERR_UNSUPPORTED, PA_OK, STATUS_NAMES, AllocStats,
                    CacheStats, PagedKVError, check, last_error, lib)
 
@@ -27,7 +27,7 @@ __all__ = [
     "PagedKVError", "lib", "STATUS_NAMES", "PA_OK", "PA_ERR_INVALID_ARG",
     "PA_ERR_OOM", "PA_ERR_NOT_FOUND", "PA_ERR_EXISTS", "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA",
     "PA_ERR_DEVICE_CHECK", "PA_DEVCHK_BLOCK_ID", "PA_DEVCHK_SLOT", "PA_DEVCHK_SEQ_LEN",
-    "PA_DEVCHK_QUERY_RANGE", "PA_DEVCHK_TIMEOUT",
+    "PA_DEVCHK_QUERY_RANGE", "PA_DEVCHK_TIMEOUT", "PA_KERNEL_DECODE", "PA_KERNEL_PREFILL",
 ]
 
 

@@ -29,6 +29,9 @@ PA_DEVCHK_SEQ_LEN = 4
 PA_DEVCHK_QUERY_RANGE = 8
 PA_DEVCHK_TIMEOUT = 16
 
+PA_KERNEL_DECODE = 1
+PA_KERNEL_PREFILL = 2
+
 STATUS_NAMES = {
     PA_OK: "ok", PA_ERR_INVALID_ARG: "invalid_arg", PA_ERR_OOM: "oom", PA_ERR_NOT_FOUND: "not_found",
     PA_ERR_EXISTS: "exists", PA_ERR_UNSUPPORTED: "unsupported", PA_ERR_CUDA: "cuda",
@@ -100,6 +103,7 @@ SIGNATURES = {
     "pa_last_error": (ctypes.c_char_p, []),
     "pa_status_string": (ctypes.c_char_p, [c_int32]),
     "pa_check_device_flag": (c_int32, [c_int32]),
+    "pa_debug_inject_stall": (c_int32, [c_int32, ctypes.c_uint64]),
     "pa_alloc_create": (c_int32, [c_int32, c_int32, _I32P, POINTER(c_void_p)]),
     "pa_alloc_destroy": (None, [_P]),
     "pa_alloc_allocate": (c_int32, [_P, c_int64, c_int32]),

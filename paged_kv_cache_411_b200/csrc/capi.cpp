@@ -46,6 +46,15 @@ const char* pa_status_string(pa_status s) {
     }
 }
 
+pa_status pa_debug_inject_stall(int32_t kernel, uint64_t wait_limit_ns) {
+    if (kernel != PA_KERNEL_DECODE && kernel != PA_KERNEL_PREFILL)
+        return fail(PA_ERR_INVALID_ARG, "pa_debug_inject_stall: kernel must be PA_KERNEL_DECODE or PA_KERNEL_PREFILL");
+    if (wait_limit_ns == 0 || wait_limit_ns > 2000000000ull)
+        return fail(PA_ERR_INVALID_ARG, "pa_debug_inject_stall: wait_limit_ns must be in 1 .. 2e9");
+    pagedkv::inject_stall(kernel == PA_KERNEL_DECODE ? pagedkv::kStallDecode : pagedkv::kStallPrefill, wait_limit_ns);
+    return PA_OK;
+}
+
 pa_status pa_check_device_flag(int32_t flag_value) {
     if (flag_value == 0) return PA_OK;
     return fail(PA_ERR_DEVICE_CHECK, "device check flag 0x%x", flag_value);

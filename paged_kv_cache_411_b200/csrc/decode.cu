@@ -103,6 +103,8 @@ struct DecodeParams {
     float* part_acc;
     int32_t max_splits;
     int32_t* err_flag;
+    uint64_t wait_ns;                   // limit of every pipeline wait (kWaitLimitNs by default)
+    int32_t stall;                      // test hook: the consumers first wait on a barrier nothing completes
 };
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -128,7 +130,7 @@ struct Cfg {
     static constexpr size_t kOffHand = kOffQ + size_t(kStages) * kQBytes;
     static constexpr size_t kOffInfo = kOffHand + size_t(2) * kHandFloats * 4;    // stage infos, then 2 hand-off infos
     static constexpr size_t kOffBar = (kOffInfo + size_t(kStages + 2) * 16 + 15) & ~size_t(15);
-    static constexpr size_t kNumBars = 3 * kStages + 4;
+    static constexpr size_t kNumBars = 3 * kStages + 5;
     static constexpr size_t kOffAbort = kOffBar + kNumBars * 8;
     static constexpr size_t kSmemBytes = kOffAbort + 16 + 1024;   // + alignment slack
     static_assert(kWPH >= 1 && kTPW >= kTPL && kTPW % kTPL == 0, "bad warp split");
@@ -348,6 +350,7 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     int4* hand_info = info + C::kStages;
     uint64_t* hand_full = empty + C::kStages;     // [2] every consumer warp has handed its state over
     uint64_t* hand_empty = hand_full + 2;         // [2] the epilogue has read the slot
+    uint64_t* never = hand_empty + 2;             // no thread ever arrives on it (failure-detection test)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffAbort);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -361,6 +364,7 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             mbar_init(&hand_full[i], kConsumerWarps);
             mbar_init(&hand_empty[i], 1);
         }
+        mbar_init(never, 1);
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -412,7 +416,7 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 const int ntok = min(kStageTok, tok0 + ntok_item - tok);
                 const int b_first = __shfl_sync(0xffffffffu, bid, tok / bs - blk0);
                 const int b_second = __shfl_sync(0xffffffffu, bid, min(tok / bs - blk0 + 1, 31));
-                if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
+                if (!mbar_wait(&empty[stage], phase ^ 1, p.wait_ns)) { ok = false; break; }
                 if (*abort_flag) { ok = false; break; }
                 if (lane == 0) {
                     int flags = ntok;
@@ -441,7 +445,7 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             nidx = __shfl_sync(0xffffffffu, nidx, 0);
             rec = nidx < n_items ? p.items[nidx] : make_int4(-1, 0, 0, 0);
         }
-        if (ok) ok = mbar_wait(&empty[stage], phase ^ 1);
+        if (ok) ok = mbar_wait(&empty[stage], phase ^ 1, p.wait_ns);
         if (!ok) {
             // Unwind: report, stop the consumers, and let every copy this warp
             // issued land before the CTA can exit (each wait again bounded).
@@ -471,7 +475,7 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         uint32_t uses = 0;
         while (true) {
             const int hs = uses & 1;
-            if (!mbar_wait(&hand_full[hs], (uses >> 1) & 1)) {
+            if (!mbar_wait(&hand_full[hs], (uses >> 1) & 1, p.wait_ns)) {
                 flag_error(p.err_flag, kDevchkTimeout);
                 *abort_flag = 1;
                 break;
@@ -528,6 +532,13 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     }
 
     // ===================================================== consumer warps
+    if (p.stall && !mbar_wait(never, 0, p.wait_ns)) {
+        // failure-detection test: the wait ran out; report it and stop the other roles, whose own
+        // waits then run out too and unwind (the producer lets its copies land before exiting)
+        flag_error(p.err_flag, kDevchkTimeout);
+        *abort_flag = 1;
+        return;
+    }
     const int hh = warp / C::kWPH;        // head within the group
     const int ww = warp % C::kWPH;        // slice of the stage's tokens
     const int tq = lane / C::kLPT;        // token row within one warp-wide load
@@ -540,13 +551,13 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     float m_run = -INFINITY, l_lane = 0.f;
     uint32_t stage = 0, phase = 0, hand_uses = 0;
     while (true) {
-        if (!mbar_wait(&full_k[stage], phase)) { flag_error(p.err_flag, kDevchkTimeout); *abort_flag = 1; break; }
+        if (!mbar_wait(&full_k[stage], phase, p.wait_ns)) { flag_error(p.err_flag, kDevchkTimeout); *abort_flag = 1; break; }
         const int4 inf = info[stage];
         const int flags = inf.w;
         if (flags & kTerminate) {
             // tell the epilogue warp there is nothing more to merge
             const int hs = hand_uses & 1;
-            if (mbar_wait(&hand_empty[hs], ((hand_uses >> 1) & 1) ^ 1)) {
+            if (mbar_wait(&hand_empty[hs], ((hand_uses >> 1) & 1) ^ 1, p.wait_ns)) {
                 if (warp == 0 && lane == 0) hand_info[hs] = make_int4(0, 0, 0, kTerminate);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&hand_full[hs]);
@@ -586,7 +597,7 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         l_lane = fmaf(l_lane, alpha, pr);
         m_run = m_new;
         // ---- P.V
-        if (!mbar_wait(&full_v[stage], phase)) { flag_error(p.err_flag, kDevchkTimeout); *abort_flag = 1; break; }
+        if (!mbar_wait(&full_v[stage], phase, p.wait_ns)) { flag_error(p.err_flag, kDevchkTimeout); *abort_flag = 1; break; }
 #pragma unroll
         for (int k = 0; k < 8; ++k) acc[k] *= alpha;
 #pragma unroll
@@ -616,7 +627,7 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             for (int off = 16; off >= 1; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
             l *= 1.0f / C::kRep;
             const int hs = hand_uses & 1;
-            if (!mbar_wait(&hand_empty[hs], ((hand_uses >> 1) & 1) ^ 1)) { flag_error(p.err_flag, kDevchkTimeout); *abort_flag = 1; break; }
+            if (!mbar_wait(&hand_empty[hs], ((hand_uses >> 1) & 1) ^ 1, p.wait_ns)) { flag_error(p.err_flag, kDevchkTimeout); *abort_flag = 1; break; }
             float* slot = hand + hs * C::kHandFloats + warp * C::kHandStride;
             if (tq == 0) {
                 *reinterpret_cast<float4*>(slot + sub * 8) = make_float4(a8[0], a8[1], a8[2], a8[3]);
@@ -699,6 +710,9 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream, const char**
     p.part_acc = reinterpret_cast<float*>(ws + w.part_acc);
     p.max_splits = w.max_splits;
     p.err_flag = a.err_flag;
+    const uint64_t stall_ns = take_injected_stall(kStallDecode);
+    p.wait_ns = stall_ns ? stall_ns : kWaitLimitNs;
+    p.stall = stall_ns != 0;
     if (a.num_seqs == 0) return cudaSuccess;
 
     const int box_tok = a.block_size >= kStageTok ? kStageTok : a.block_size;

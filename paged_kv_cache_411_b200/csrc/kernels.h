@@ -60,4 +60,13 @@ bool encode_tensor_map_3d(void* map_out, const void* base, uint64_t d0, uint64_t
 
 int32_t device_sm_count();
 
+// Failure-detection test hook (pa_debug_inject_stall): the next launch of the given kernel
+// (kStallDecode / kStallPrefill) gets this pipeline-wait limit and makes its consumer role wait on a
+// barrier nothing completes.  Returns 0 (no stall; the default limit) or the limit in ns, and
+// clears the request.
+constexpr int32_t kStallDecode = 1;
+constexpr int32_t kStallPrefill = 2;
+uint64_t take_injected_stall(int32_t kernel);
+void inject_stall(int32_t kernel, uint64_t limit_ns);
+
 }  // namespace pagedkv

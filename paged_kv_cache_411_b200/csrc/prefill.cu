@@ -69,6 +69,8 @@ struct PrefillParams {
     int32_t B, T, H, max_blocks, bs, num_blocks, grid_tiles, box_rows;
     float qscale;
     int32_t* err_flag;
+    uint64_t wait_ns;          // limit of every pipeline wait (kWaitLimitNs by default)
+    int32_t stall;             // test hook: the softmax warps first wait on a barrier nothing completes
 };
 
 template <int D>
@@ -81,7 +83,7 @@ struct PCfg {
     static constexpr size_t kOffK = kOffQ + kOpBytes;
     static constexpr size_t kOffV = kOffK + size_t(kStages) * kOpBytes;
     static constexpr size_t kOffBar = kOffV + size_t(kStages) * kOpBytes;
-    static constexpr int kNumBars = 12;
+    static constexpr int kNumBars = 13;
     static constexpr size_t kOffSlot = kOffBar + kNumBars * 8;
     static constexpr size_t kOffRed = kOffSlot + 64;                 // final exchange: maxes [2][128], sums [2][128]
     // Every CTA takes all 512 TMEM columns, so the request is kept above half the SM's shared
@@ -118,6 +120,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint64_t* pv_done = bars + 8;    // [2] P.V(j) has landed in O_0/O_1, which also frees V stage j % 2
     uint64_t* drain = bars + 10;
     uint64_t* sum_bar = bars + 11;   // final (max, sum) exchange between the two halves of a row
+    uint64_t* never = bars + 12;     // no thread ever arrives on it (failure-detection test)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffSlot);
     volatile int* info = reinterpret_cast<volatile int*>(smem + C::kOffSlot + 16);   // b, qt, abort
 
@@ -159,6 +162,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         mbar_init(p_full, kSoftmaxWarps);
         mbar_init(drain, 1);
         mbar_init(sum_bar, kSoftmaxWarps);
+        mbar_init(never, 1);
         mbar_init_fence();
     }
     __syncthreads();
@@ -227,7 +231,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int bid_next = read_id(j + 1);
             const int n_mine = (nbox * C::kChunks - wsub + kIssueWarps - 1) / kIssueWarps;
             const uint32_t bytes = static_cast<uint32_t>(n_mine * br * 128);
-            if (!mbar_wait(&empty[st], ((j >> 1) & 1) ^ 1)) { abort_now(); break; }
+            if (!mbar_wait(&empty[st], ((j >> 1) & 1) ^ 1, p.wait_ns)) { abort_now(); break; }
             if (info[2]) break;
             if (lane == 0) mbar_arrive_expect_tx(&full[st], bytes);
             __syncwarp();
@@ -257,13 +261,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const uint64_t dQ = umma_desc_sw128(smem_u32(sQ), 16, 1024);
             const uint64_t dK = umma_desc_sw128(smem_u32(sK), 16, 1024);
             const uint64_t dV = umma_desc_sw128(smem_u32(sV), C::kChunkBytes, 1024);
-            bool ok = mbar_wait(q_full, 0);
+            bool ok = mbar_wait(q_full, 0, p.wait_ns);
             // An mbarrier answers after ~150 cycles even when its phase is complete, so this thread asks
             // early (mbar_test_wait) and collects the answers after the MMAs it issues meanwhile; it only
             // blocks when a phase really is still open.
             auto issue_s = [&](int j, bool k_ready) -> bool {
                 const int st = j & 1;
-                if (!k_ready && !mbar_wait(&k_full[st], (j >> 1) & 1)) return false;
+                if (!k_ready && !mbar_wait(&k_full[st], (j >> 1) & 1, p.wait_ns)) return false;
                 // S(j) reuses the buffer of S(j-2)/P(j-2): it is issued after P.V(j-2), which the
                 // tensor core runs first, and P.V(j-2) waited for every softmax warp to finish that tile
                 tc_fence_after_sync();
@@ -284,8 +288,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const bool p_ready = mbar_test_wait(p_full, j & 1);
                 const bool v_ready = mbar_test_wait(&v_full[st], (j >> 1) & 1);
                 if (j + 1 < n_tiles && !(ok = issue_s(j + 1, k_ready))) break;
-                if (!p_ready && !(ok = mbar_wait(p_full, j & 1))) break;
-                if (!v_ready && !(ok = mbar_wait(&v_full[st], (j >> 1) & 1))) break;
+                if (!p_ready && !(ok = mbar_wait(p_full, j & 1, p.wait_ns))) break;
+                if (!v_ready && !(ok = mbar_wait(&v_full[st], (j >> 1) & 1, p.wait_ns))) break;
                 if (info[2]) { ok = false; break; }
                 k_ready = j + 2 < n_tiles && mbar_test_wait(&k_full[st], ((j + 2) >> 1) & 1);   // for S(j+2)
                 tc_fence_after_sync();
@@ -323,9 +327,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const uint32_t o_mine = lane_base + C::kColO + g * D;
         const float qs = p.qscale;
         float m = -INFINITY, l = 0.f;                    // log2-domain running max and sum of this half
-        bool ok = true;
+        // failure-detection test: the wait runs out and the softmax role stops; the MMA issuer and the
+        // producers then run out of their own waits and unwind
+        bool ok = !p.stall || mbar_wait(never, 0, p.wait_ns);
         for (int j = 0; j < n_tiles && ok; ++j) {
-            if (!(ok = mbar_wait(&s_full[j & 1], (j >> 1) & 1))) break;
+            if (!(ok = mbar_wait(&s_full[j & 1], (j >> 1) & 1, p.wait_ns))) break;
             tc_fence_after_sync();
             const int key0 = j * kTile;
             const bool diag = key0 + kTile - 1 > tile_pos0;          // some key of the tile is masked
@@ -371,7 +377,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             l = fmaf(l, alpha, (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
             if (j > 0 && __any_sync(0xffffffffu, raise)) {
                 // O_g holds the sum up to tile j-1: wait for that P.V, then rescale this warp's rows
-                if (!(ok = mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1))) break;
+                if (!(ok = mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, p.wait_ns))) break;
                 tc_fence_after_sync();
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
@@ -388,7 +394,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tmem_wait_st();
             if (j == n_tiles - 1 && kv_len < key0 + kTile) {
                 // rows of V past the sequence end may hold anything: zero them before P.V reads them
-                if (!(ok = mbar_wait(&v_full[j & 1], (j >> 1) & 1))) break;
+                if (!(ok = mbar_wait(&v_full[j & 1], (j >> 1) & 1, p.wait_ns))) break;
                 if (key0 + r >= kv_len) {
                     uint8_t* vrow = sV + (j & 1) * C::kOpBytes + r * 128;
 #pragma unroll
@@ -410,8 +416,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         red[256 + g * 128 + r] = l;
         __syncwarp();
         if (lane == 0) mbar_arrive(sum_bar);
-        if (ok) ok = mbar_wait(sum_bar, 0);
-        if (ok) ok = mbar_wait(&pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1);   // the last P.V has landed
+        if (ok) ok = mbar_wait(sum_bar, 0, p.wait_ns);
+        if (ok) ok = mbar_wait(&pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, p.wait_ns);   // the last P.V has landed
         if (ok) {
             tc_fence_after_sync();
             const float m0 = red[r], m1 = red[128 + r];
@@ -499,6 +505,9 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream, const char
     p.box_rows = br;
     p.qscale = a.scale * kLog2eP;
     p.err_flag = a.err_flag;
+    const uint64_t stall_ns = take_injected_stall(kStallPrefill);
+    p.wait_ns = stall_ns ? stall_ns : kWaitLimitNs;
+    p.stall = stall_ns != 0;
     const dim3 grid(p.grid_tiles, a.num_heads);
     if (a.head_dim == 128) return run_prefill<128>(tq, tk, tv, p, grid, stream);
     return run_prefill<64>(tq, tk, tv, p, grid, stream);

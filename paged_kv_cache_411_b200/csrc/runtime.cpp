@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "kernels.h"
@@ -62,5 +63,11 @@ int32_t device_sm_count() {
     }
     return cache[dev];
 }
+
+static std::atomic<uint64_t> g_stall_ns[3];
+
+void inject_stall(int32_t kernel, uint64_t limit_ns) { g_stall_ns[kernel].store(limit_ns); }
+
+uint64_t take_injected_stall(int32_t kernel) { return g_stall_ns[kernel].exchange(0); }
 
 }  // namespace pagedkv

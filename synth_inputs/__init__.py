@@ -211,12 +211,20 @@ def long_shared_prefix() -> Workload:
                     shared_prefix=1024)
 
 
+def causal_prefill_8k() -> Workload:
+    """One 8192-token prompt prefilled as a single causal chunk (nothing cached before it)."""
+    return Workload(name="llama2_7b_prefill8192_causal_bs16", seed=6, num_heads=32, head_dim=128,
+                    block_size=16, decode_lens=(), pool_factor=1.1,
+                    prefill=PrefillSpec(ctx_before=0, chunk=8192))
+
+
 WORKLOADS = {
     "tiny": tiny,
     "b32": llama7b_b32,
     "b256": llama7b_b256_ragged,
     "mixed": mixed_prefill_decode,
     "longctx": long_shared_prefix,
+    "prefill8k": causal_prefill_8k,
 }
 
 

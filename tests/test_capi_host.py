@@ -227,3 +227,10 @@ def test_internal_waste_matches_page_estimate(bs):
     _, t, lens = r.alloc.pack(np.arange(S), max(-(-n // bs) for n in w.decode_lens))
     waste = (t >= 0).sum(axis=1) * bs - lens
     assert (waste >= 0).all() and (waste < bs).all() and waste.sum() == st["waste_tokens"]
+
+
+def test_stall_hook_arguments():
+    lib = pk.lib()
+    assert lib.pa_debug_inject_stall(3, 1000) == pk.PA_ERR_INVALID_ARG
+    assert lib.pa_debug_inject_stall(pk.PA_KERNEL_DECODE, 0) == pk.PA_ERR_INVALID_ARG
+    assert lib.pa_debug_inject_stall(pk.PA_KERNEL_PREFILL, 3_000_000_000) == pk.PA_ERR_INVALID_ARG

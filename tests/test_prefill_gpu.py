@@ -184,3 +184,31 @@ def test_prefill_many_requests(cuda_ready):
     assert np.isfinite(out).all()
     diff = np.abs(out - ref)
     assert diff.max() <= TOL, f"max abs error {diff.max():.3g}"
+
+
+def test_causal_prefill_8192_every_row(cuda_ready):
+    """The 8192-token causal prefill the benchmark times (one request, nothing cached, 32 heads x 128),
+    in the bench's launch configuration.  Every row of every head is compared with the oracle, which
+    computes the prompt as 256-row chunks at their absolute positions (the chunk-split identity its
+    pins establish), so its float64 score matrices stay within host memory."""
+    w = si.get("prefill8k")
+    ds = pwl.build(w)
+    pk.reshape_and_cache(ds.k_step, ds.v_step, ds.k_cache, ds.v_cache, ds.slot_mapping)
+    out = torch.full_like(ds.prefill_q, float("nan"))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pk.paged_attention_prefill_chunk(out, ds.prefill_q, ds.k_cache, ds.v_cache, ds.prefill_table,
+                                     ds.prefill_q_start, ds.prefill_ctx_before, w.scale, err_flag=err)
+    got = out.float().cpu().numpy()
+    assert int(err.item()) == 0
+    o = owl.build(w)
+    kc, vc = o.k_cache.copy(), o.v_cache.copy()
+    oatt.reshape_and_cache(kc, vc, o.k_step, o.v_step, o.slot_mapping, w.block_size)
+    assert np.array_equal(ds.k_cache.cpu().numpy().view(np.int16), kc.view(np.int16))
+    L, step = w.prefill.chunk, 256
+    worst = 0.0
+    for lo in range(0, L, step):
+        hi = min(L, lo + step)
+        ref = oatt.paged_attention_prefill_chunk(o.prefill_q[lo:hi], kc, vc, o.prefill_table, [0, hi - lo], [lo],
+                                                 w.block_size, w.scale)
+        worst = max(worst, float(np.abs(got[lo:hi] - ref).max()))
+    assert worst <= TOL, f"max abs error {worst:.3g}"
