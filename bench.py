@@ -59,6 +59,22 @@ def prefill_flops(w):
     return 4 * w.num_heads * w.head_dim * pairs
 
 
+def shared_prefix_rereads(w, seq_lens):
+    """K/V bytes the decode reads more than once: a prefix shared by all sequences (whole blocks) is
+    stored once but every sequence reads it, so its bytes beyond the first read are not unique."""
+    if not w.shared_prefix or len(seq_lens) == 0:
+        return 0
+    shared_tokens = (w.shared_prefix // w.block_size) * w.block_size
+    return (len(seq_lens) - 1) * shared_tokens * w.num_heads * w.head_dim * 2 * 2
+
+
+def dist_ms(xs):
+    """Median, 10th and 90th percentile (and mean) of per-step times in ms."""
+    a = np.asarray(xs, dtype=np.float64)
+    return {"median": round(float(np.median(a)), 5), "p10": round(float(np.percentile(a, 10)), 5),
+            "p90": round(float(np.percentile(a, 90)), 5), "mean": round(float(a.mean()), 5), "n": int(a.size)}
+
+
 def step_bytes(w, seq_lens, tables_cols, n_step_rows):
     """Algorithmic bytes of one step (see the module docstring)."""
     H, D, bs = w.num_heads, w.head_dim, w.block_size
@@ -244,6 +260,35 @@ def _blas_threads():
         return os.cpu_count() or 1
 
 
+def time_oracle_prefill(w, steps, target_seconds):
+    """Times the oracle's causal prefill on the chunk's last rows (the heaviest ones), as many rows as fit
+    about target_seconds over all steps.  Returns (step GB/s estimated from the sampled share of the
+    chunk's FLOPs, seconds per sampled call, description, threads)."""
+    from oracle import attention as oatt
+    from oracle import workloads as owl
+    o = owl.build(w)
+    kc, vc = o.k_cache.copy(), o.v_cache.copy()
+    oatt.reshape_and_cache(kc, vc, o.k_step, o.v_step, o.slot_mapping, w.block_size)
+    L, c = w.prefill.chunk, w.prefill.ctx_before
+
+    def call(rows):
+        lo = L - rows
+        t0 = time.perf_counter()
+        oatt.paged_attention_prefill_chunk(o.prefill_q[lo:], kc, vc, o.prefill_table, [0, rows], [c + lo],
+                                           w.block_size, w.scale)
+        return time.perf_counter() - t0
+
+    rows = max(1, min(L, int(16 * target_seconds / max(1, steps) / max(call(16), 1e-6))))
+    dts = [call(rows) for _ in range(steps)]
+    dt = float(np.mean(dts))
+    pairs = rows * c + sum(L - i for i in range(rows))               # visible (query, key) pairs sampled
+    share = pairs / (L * c + L * (L + 1) // 2)
+    _, rs_b, pre_b = step_bytes(w, [], 0, o.slot_mapping.shape[0])
+    desc = (f"oracle float64 causal prefill of the last {rows} of {L} rows ({100 * share:.2f}% of the chunk's "
+            f"FLOPs) per step, {steps} timed steps; GB/s = the step's bytes over the time scaled to the whole chunk")
+    return (rs_b + pre_b) / (dt / share) / 1e9, dt, desc, _blas_threads()
+
+
 def run_reference(args):
     world, rank, _ = dist_setup()
     if rank != 0:
@@ -251,6 +296,20 @@ def run_reference(args):
     w = si.get(args.workload)
     if args.block_size:
         w = si.with_block_size(w, args.block_size)
+    if w.num_seqs == 0:
+        gbs, dt, desc, threads = time_oracle_prefill(w, args.steps, 120.0)
+        line = {
+            "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "num_heads": w.num_heads, "head_dim": w.head_dim,
+                       "block_size": w.block_size, "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return 0
     per_step = oracle_tokens_for(w, args.steps + args.warmup, 120.0)
     gbs, dt, desc, threads = time_oracle(w, args.steps, args.warmup, per_step)
     line = {
@@ -304,6 +363,8 @@ def run_ours(args):
                                              ds.prefill_q_start, ds.prefill_ctx_before, w.scale, stream=stream)
             if pev is not None:
                 pev[1].record(stream)
+        if S == 0:
+            return
         if ev is not None:
             ev[0].record(stream)
         pk.paged_attention_decode(out, ds.q, ds.k_cache, ds.v_cache, ds.block_tables, ds.seq_lens, w.scale, ws,
@@ -317,6 +378,7 @@ def run_ours(args):
 
     dec_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                   for _ in range(args.steps)]
+    step_events = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     pre_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                   for _ in range(args.steps)] if pout is not None else [None] * args.steps
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -327,13 +389,16 @@ def run_ours(args):
         torch.cuda.synchronize(device)
         t0.record(stream)
         for i in range(args.steps):
+            step_events[i].record(stream)
             step(dec_events[i], pre_events[i])
+        step_events[args.steps].record(stream)
         t1.record(stream)
         torch.cuda.synchronize(device)
         if world > 1:
             dist.barrier()
     local_ms = t0.elapsed_time(t1)
-    dec_ms = [a.elapsed_time(b) for a, b in dec_events]
+    dec_ms = [a.elapsed_time(b) for a, b in dec_events] if S > 0 else []
+    step_ms = [step_events[i].elapsed_time(step_events[i + 1]) for i in range(args.steps)]
     pre_ms = [e[0].elapsed_time(e[1]) for e in pre_events] if pout is not None else []
     total_ms, total_bytes = reduce_max_sum(local_ms, step_b * args.steps, device)
     ms_per_step = total_ms / args.steps
@@ -348,11 +413,12 @@ def run_ours(args):
     if pout is not None:
         names += ("prefill_q", "prefill_table", "prefill_q_start", "prefill_ctx_before")
     host = {k: getattr(ds, k).cpu().pin_memory() for k in names}
-    host_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    outs = [out] + ([pout] if pout is not None else [])
+    host_out = [[torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs] for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = host_out[0].numel() * host_out[0].element_size()
+    d2h = sum(t.numel() * t.element_size() for t in host_out[0])
     dev_in = [{k: torch.empty_like(getattr(ds, k)) for k in names} for _ in range(2)]
-    dev_out = [torch.empty_like(out) for _ in range(2)]
+    dev_out = [[torch.empty_like(o) for o in outs] for _ in range(2)]
     copy_stream = torch.cuda.Stream(device)
     ready = [torch.cuda.Event() for _ in range(2)]      # inputs of the set are on the device
     done = [torch.cuda.Event() for _ in range(2)]       # the step that used the set has finished
@@ -370,14 +436,17 @@ def run_ours(args):
         stream.wait_event(ready[b])
         pk.reshape_and_cache(d["k_step"], d["v_step"], ds.k_cache, ds.v_cache, d["slot_mapping"], stream=stream)
         if pout is not None:
-            pk.paged_attention_prefill_chunk(pout, d["prefill_q"], ds.k_cache, ds.v_cache, d["prefill_table"],
-                                             d["prefill_q_start"], d["prefill_ctx_before"], w.scale, stream=stream)
-        pk.paged_attention_decode(dev_out[b], d["q"], ds.k_cache, ds.v_cache, d["block_tables"], d["seq_lens"],
-                                  w.scale, ws, stream=stream)
+            pk.paged_attention_prefill_chunk(dev_out[b][1], d["prefill_q"], ds.k_cache, ds.v_cache,
+                                             d["prefill_table"], d["prefill_q_start"], d["prefill_ctx_before"],
+                                             w.scale, stream=stream)
+        if S > 0:
+            pk.paged_attention_decode(dev_out[b][0], d["q"], ds.k_cache, ds.v_cache, d["block_tables"],
+                                      d["seq_lens"], w.scale, ws, stream=stream)
         done[b].record(stream)
         with torch.cuda.stream(copy_stream):
             copy_stream.wait_event(done[b])
-            host_out[b].copy_(dev_out[b], non_blocking=True)
+            for h, dv in zip(host_out[b], dev_out[b]):
+                h.copy_(dv, non_blocking=True)
             fetched[b].record(copy_stream)
 
     def e2e_run(n):
@@ -404,8 +473,10 @@ def run_ours(args):
     e2e_value = e2e_bytes / e2e_max / 1e9
 
     if rank == 0:
-        dec_avg_ms = float(np.mean(dec_ms))
-        dec_gbs = dec_b / (dec_avg_ms / 1e3) / 1e9
+        has_decode = S > 0
+        dec_avg_ms = float(np.mean(dec_ms)) if has_decode else 0.0
+        unique_b = dec_b - shared_prefix_rereads(w, ds.seq_lens_host)
+        dec_gbs = unique_b / (dec_avg_ms / 1e3) / 1e9 if has_decode else 0.0
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
@@ -424,25 +495,42 @@ def run_ours(args):
             "roofline": {"kernel": "paged_attention_decode (plan + streaming kernel + combine)", "bound": "hbm",
                          "achieved": round(dec_gbs, 2), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": round(dec_gbs / peak, 4), "traffic": ncu_traffic(w, args, "decode"),
-                         "algorithmic_bytes_per_launch": dec_b, "avg_launch_ms": round(dec_avg_ms, 5)},
+                         "algorithmic_bytes_per_launch": unique_b, "avg_launch_ms": round(dec_avg_ms, 5)},
+            "step_ms": dist_ms(step_ms),
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(1e3 * e2e_max / args.steps, 4)},
-            "gpu_launches": args.steps * (4 + (1 if pout is not None else 0)),
+            "gpu_launches": args.steps * (1 + (3 if S > 0 else 0) + (1 if pout is not None else 0)),
             "kv_pool": pool_stats(ds),
             "clocks": clk.summary(),
         }
+        if has_decode:
+            line["decode_ms"] = dist_ms(dec_ms)
+            if unique_b != dec_b:
+                # a shared prefix is read by every sequence but stored once: the roofline counts it once
+                line["roofline"]["logical_bytes_per_launch"] = dec_b
+                line["roofline"]["logical_achieved"] = round(dec_b / (dec_avg_ms / 1e3) / 1e9, 2)
         if pout is not None:
             pre_avg = float(np.mean(pre_ms))
             tf = prefill_flops(w) / (pre_avg / 1e3) / 1e12
+            line["prefill_ms"] = dist_ms(pre_ms)
             line["roofline_prefill"] = {
                 "kernel": "paged_attention_prefill_chunk (tcgen05)", "bound": "tensor", "achieved": round(tf, 2),
                 "peak": peak_tf, "peak_kind": peak_kind + " bf16 burst (fp16 has the same nominal rate)",
                 "unit": "TFLOP/s", "frac": round(tf / peak_tf, 4), "traffic": ncu_traffic(w, args, "prefill"),
                 "algorithmic_flops_per_launch": prefill_flops(w), "avg_launch_ms": round(pre_avg, 5)}
-        if world == 1 and not args.no_cpu_baseline:
+            if not has_decode:
+                # a prefill-only step: its tensor-bound kernel is the dominant one
+                line["roofline"] = line.pop("roofline_prefill")
+        if world == 1 and not args.no_cpu_baseline and has_decode:
             gbs, dt, desc, threads = time_oracle(w, 1, 1, args.oracle_tokens, min_seconds=10.0, max_steps=30)
             line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
                                     "sample": desc}
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1, user_api="blas"):
+                gbs1, _, desc1, threads1 = time_oracle(w, 1, 1, args.oracle_tokens // 4, min_seconds=10.0,
+                                                       max_steps=30)
+            line["cpu_baseline_1thread"] = {"value": round(gbs1, 4), "unit": "GB/s", "cores": threads1,
+                                            "kind": "oracle", "sample": desc1}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -522,13 +610,17 @@ def run_serve(args):
         if T:
             slots = stage("slots", plan["slot_mapping"])
             if P:
-                alloc.pack(plan["prefill_reqs"], mb, tables=host_v["pt"][:P])     # straight into staging
+                st, _, _ = alloc.pack(plan["prefill_reqs"], mb, tables=host_v["pt"][:P])   # straight into staging
+                if st != pk.PA_OK:
+                    raise SystemExit(f"serve: packing the prefill tables failed: {pk.last_error()}")
                 q_start = np.concatenate([[0], np.cumsum(plan["prefill_len"])]).astype(np.int32)
                 pt_d = dev_v["pt"][:P]
                 qs_d = stage("qs", q_start)
                 ctx_d = stage("ctx", plan["prefill_ctx"])
             if S:
-                alloc.pack(plan["decode_reqs"], mb, tables=host_v["dt"][:S], lens=host_v["dl"][:S])
+                st, _, _ = alloc.pack(plan["decode_reqs"], mb, tables=host_v["dt"][:S], lens=host_v["dl"][:S])
+                if st != pk.PA_OK:
+                    raise SystemExit(f"serve: packing the decode tables failed: {pk.last_error()}")
                 dt_d, dl_d = dev_v["dt"][:S], dev_v["dl"][:S]
             dev_buf.copy_(host_buf, non_blocking=True)       # the step's inputs, one copy
             host_s += time.perf_counter() - h0

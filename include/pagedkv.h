@@ -294,7 +294,7 @@ typedef struct {
 } pa_step_info_t;
 
 typedef struct {
-    int32_t state;              /* 0 waiting, 1 running, 2 finished                   */
+    int32_t state;              /* 0 waiting, 1 running, 2 finished, 3 swapped out    */
     int32_t prompt_len;
     int32_t max_new_tokens;
     int32_t prefilled;          /* tokens of the current prefill already cached       */
@@ -308,6 +308,8 @@ typedef struct {
 
 typedef struct {
     int64_t steps, waiting, running, finished, preemptions, prefill_tokens, decode_tokens;
+    int64_t swapped;            /* requests swapped out now                           */
+    int64_t swap_outs, swap_ins;  /* moves so far                                     */
 } pa_sched_stats_t;
 
 /* Errors: INVALID_ARG (NULL, non-positive caps, negative watermark). */
@@ -332,6 +334,29 @@ pa_status pa_sched_step(pa_sched* s, pa_step_info_t* info, int64_t* prefill_reqs
  * that emitted max_new_tokens finishes (freed at the next step).
  * Errors: INVALID_ARG (no open step). */
 pa_status pa_sched_complete(pa_sched* s);
+
+/* Swap preemption ([CB-PA] §5.4 strategy 2 "Swap to CPU", §4.4 SwappingManager).
+ * With a CPU-side allocator attached (same block_size; NULL detaches, allowed
+ * only while nothing is swapped out), a preempted request is moved to the CPU
+ * pool (pa_alloc_swap_out bookkeeping, no data moved by the scheduler) instead
+ * of being freed, keeping its progress; if the CPU pool cannot take it, it is
+ * recomputed as without swapping.  Each step first brings swapped requests
+ * back (most recently preempted first) while seats are free and the blocks of
+ * their table, plus one if their next decode opens a block, plus the
+ * decodes' needs and the watermark are available, and admits no waiting
+ * request while one is still swapped out.  The allocator is borrowed and must
+ * outlive the scheduler.  Errors: INVALID_ARG (NULL scheduler, block sizes
+ * differ, a step is open, detaching while requests are swapped out). */
+pa_status pa_sched_enable_swap(pa_sched* s, pa_alloc* cpu);
+/* The block moves of the last scheduled step, which the caller performs before
+ * the step's kernels, swap-outs first (e.g. pa_swap_blocks GPU -> CPU pool,
+ * then CPU -> GPU): out_pairs[2i], out_pairs[2i+1] = (GPU block, CPU block) of
+ * a swap-out; in_pairs likewise (CPU block, GPU block).  Host int64 arrays of
+ * capacity out_cap / in_cap pairs (either may be NULL); *n_out / *n_in
+ * (nullable) = the pair counts.  Errors: INVALID_ARG (NULL scheduler; a
+ * capacity below its count, nothing copied). */
+pa_status pa_sched_last_swaps(const pa_sched* s, int64_t* out_pairs, int32_t out_cap, int32_t* n_out,
+                              int64_t* in_pairs, int32_t in_cap, int32_t* n_in);
 pa_status pa_sched_request_info(const pa_sched* s, int64_t req, pa_request_info_t* out);
 pa_status pa_sched_stats(const pa_sched* s, pa_sched_stats_t* out);
 

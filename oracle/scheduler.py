@@ -22,6 +22,22 @@ loop.  Readings where the sketch leaves a step open:
   rows, then the decode rows;
 * finishing: a request emits a token when its prefill completes and at each
   decode; at ``max_new_tokens`` it finishes and is freed at the next step.
+
+§5.4 also names a second preemption strategy, swapping the victim's KV to CPU
+memory (§4.4's ``SwappingManager``).  With a CPU block manager given
+(``swap_cpu``), a victim is moved to the CPU pool instead of being freed
+(``oracle.swap``: destination allocated first, block i to block i, source
+freed); when the CPU pool cannot take it, it is recomputed as above.  Readings
+where the page leaves the strategy open:
+
+* a swapped request keeps its progress (prefilled and generated tokens) and
+  waits in a swapped queue, the most recently preempted at the front;
+* swapped requests come back before any waiting request is admitted, in queue
+  order, while seats are free and the blocks of their table (plus one if their
+  next decode opens a block), the decodes' needs and the watermark are
+  available; no waiting request is admitted while a request is still swapped;
+* the step reports its block moves (GPU to CPU for the swap-outs, then CPU to
+  GPU for the swap-ins), which the caller performs before the step's kernels.
 """
 from __future__ import annotations
 
@@ -29,8 +45,9 @@ from collections import deque
 
 from .block_manager import OK, OOM
 from .sizes import blocks_needed
+from .swap import SwappingManager
 
-WAITING, RUNNING, FINISHED = 0, 1, 2
+WAITING, RUNNING, FINISHED, SWAPPED = 0, 1, 2, 3
 
 
 class _Req:
@@ -47,8 +64,13 @@ class _Req:
 
 
 class Scheduler:
-    def __init__(self, bm, max_num_seqs, max_num_tokens, chunked_prefill=True, watermark_blocks=0):
+    def __init__(self, bm, max_num_seqs, max_num_tokens, chunked_prefill=True, watermark_blocks=0,
+                 swap_cpu=None):
         self.bm = bm
+        self.swapper = SwappingManager(bm, swap_cpu) if swap_cpu is not None else None
+        self.swapped: deque = deque()
+        self.swap_out_pairs: list = []
+        self.swap_in_pairs: list = []
         self.max_num_seqs = max_num_seqs
         self.max_num_tokens = max_num_tokens
         self.chunked = bool(chunked_prefill)
@@ -75,16 +97,20 @@ class Scheduler:
 
     def step(self):
         info = dict(step=self.steps, num_admitted=0, num_preempted=0, num_finished=0)
+        self.swap_out_pairs, self.swap_in_pairs = [], []
         self._free_finished(info)
         need = self._preempt(info)
-        self._admit(info, need)
+        need = self._swap_in(info, need)
+        if not self.swapped:
+            self._admit(info, need)
         self.last_prefill, self.last_decode = [], []
         dec_slots = self._schedule_decodes()
         pre_slots = self._schedule_prefills(self.max_num_tokens)
         info.update(num_prefill=len(self.last_prefill), num_decode=len(self.last_decode),
                     num_tokens=len(pre_slots) + len(dec_slots),
                     prefill=list(self.last_prefill), decode=list(self.last_decode),
-                    slot_mapping=pre_slots + dec_slots)
+                    slot_mapping=pre_slots + dec_slots, swap_out=list(self.swap_out_pairs),
+                    swap_in=list(self.swap_in_pairs))
         return info
 
     # §2.2 step 1: requests that emitted their last token give their blocks back
@@ -98,20 +124,48 @@ class Scheduler:
                 keep.append(r)
         self.running = keep
 
-    # §5.4 strategy 1: preempt the newest running request while the decodes lack blocks
+    # §5.4: preempt the newest running request while the decodes lack blocks; strategy 2 (swap its KV
+    # to the CPU pool) when a CPU pool is given and has room, else strategy 1 (recompute)
     def _preempt(self, info):
         need = self._need()
         while need > self.bm._available() and self.running:
             v = self.running.pop()
             q = self.reqs[v]
+            q.preemptions += 1
+            info["num_preempted"] += 1
+            if self.swapper is not None:
+                gpu_table = list(self.bm.block_tables[v])
+                if self.swapper.swap_out(v) == OK:
+                    self.swap_out_pairs += list(zip(gpu_table, self.swapper.cpu.block_tables[v]))
+                    q.state = SWAPPED
+                    self.swapped.appendleft(v)
+                    need = self._need()
+                    continue
             self.bm.free(v)
             q.to_prefill = q.prompt_len + q.generated
             q.prefilled = 0
             q.state = WAITING
-            q.preemptions += 1
             self.waiting.appendleft(v)
-            info["num_preempted"] += 1
             need = self._need()
+        return need
+
+    # swapped requests come back first (§4.4 swap_in), while seats and blocks last
+    def _swap_in(self, info, need):
+        bs = self.bm.block_size
+        while self.swapped and len(self.running) < self.max_num_seqs:
+            r = self.swapped[0]
+            q = self.reqs[r]
+            cpu_table = list(self.swapper.cpu.block_tables[r])
+            opens = 1 if (q.prefilled == q.to_prefill and q.generated < q.max_new
+                          and self.swapper.cpu.seq_lens[r] % bs == 0) else 0
+            if self.bm._available() - need - self.watermark < len(cpu_table) + opens:
+                break
+            self.swapped.popleft()
+            assert self.swapper.swap_in(r) == OK
+            self.swap_in_pairs += list(zip(cpu_table, self.bm.block_tables[r]))
+            q.state = RUNNING
+            self.running.append(r)
+            need += opens
         return need
 
     # §2.2 step 2 with §5.3's watermark: admit in arrival order while seats and blocks last

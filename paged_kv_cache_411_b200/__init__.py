@@ -112,8 +112,10 @@ class BlockAllocator:
         if lens is None:
             lens = np.empty(n, dtype=np.int32)
         if (tables.dtype != np.int32 or tables.shape != (n, max_blocks) or not tables.flags.c_contiguous
-                or lens.dtype != np.int32 or lens.shape != (n,) or not lens.flags.c_contiguous):
-            raise ValueError("pack: tables must be int32 [n, max_blocks] and lens int32 [n], C-contiguous")
+                or not tables.flags.writeable or lens.dtype != np.int32 or lens.shape != (n,)
+                or not lens.flags.c_contiguous or not lens.flags.writeable):
+            raise ValueError("pack: tables must be int32 [n, max_blocks] and lens int32 [n], C-contiguous and "
+                             "writeable")
         st = lib().pa_alloc_pack(self._h, _i64p(r), n, max_blocks, _i32p(tables), _i32p(lens))
         return st, tables, lens
 
@@ -168,6 +170,7 @@ class Scheduler:
                  watermark_blocks: int = 0):
         from ._lib import SchedConfig
         self._alloc = alloc                       # the C scheduler borrows it
+        self._cpu = None
         self.max_num_seqs, self.max_num_tokens = int(max_num_seqs), int(max_num_tokens)
         cfg = SchedConfig(self.max_num_seqs, self.max_num_tokens, int(bool(chunked_prefill)), int(watermark_blocks))
         self._h = c_void_p()
@@ -203,7 +206,25 @@ class Scheduler:
         P, D, T = info.num_prefill, info.num_decode, info.num_tokens
         d.update(prefill_reqs=pr[:P].copy(), prefill_ctx=pc[:P].copy(), prefill_len=pl[:P].copy(),
                  decode_reqs=dr[:D].copy(), decode_seq_lens=dl[:D].copy(), slot_mapping=sm[:T].copy())
+        if self._cpu is not None:
+            d["swap_out"], d["swap_in"] = self.last_swaps()
         return d
+
+    def enable_swap(self, cpu: "BlockAllocator") -> int:
+        """Preempt by swapping to `cpu` (a BlockAllocator over the host pool; None: recompute)."""
+        st = lib().pa_sched_enable_swap(self._h, None if cpu is None else cpu._h)
+        if st == PA_OK:
+            self._cpu = cpu                       # the C scheduler borrows it
+        return st
+
+    def last_swaps(self):
+        """Block moves of the last step: (swap-out pairs [n, 2] GPU -> CPU, swap-in pairs [m, 2] CPU -> GPU)."""
+        no, ni = c_int32(0), c_int32(0)
+        check(lib().pa_sched_last_swaps(self._h, None, 0, byref(no), None, 0, byref(ni)))
+        out = np.empty((no.value, 2), np.int64)
+        inn = np.empty((ni.value, 2), np.int64)
+        check(lib().pa_sched_last_swaps(self._h, _i64p(out), no.value, byref(no), _i64p(inn), ni.value, byref(ni)))
+        return out, inn
 
     def complete(self) -> None:
         check(lib().pa_sched_complete(self._h))

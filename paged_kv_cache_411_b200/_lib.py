@@ -87,7 +87,7 @@ class RequestInfo(ctypes.Structure):
 
 class SchedStats(ctypes.Structure):
     _fields_ = [(k, c_int64) for k in ("steps", "waiting", "running", "finished", "preemptions",
-                                        "prefill_tokens", "decode_tokens")]
+                                        "prefill_tokens", "decode_tokens", "swapped", "swap_outs", "swap_ins")]
 
     def as_dict(self):
         return {k: getattr(self, k) for k, _ in self._fields_}
@@ -130,6 +130,8 @@ SIGNATURES = {
     "pa_sched_add_request": (c_int32, [_P, c_int64, c_int32, c_int32]),
     "pa_sched_step": (c_int32, [_P, POINTER(StepInfo), _I64P, _I32P, _I32P, _I64P, _I32P, _I64P]),
     "pa_sched_complete": (c_int32, [_P]),
+    "pa_sched_enable_swap": (c_int32, [_P, _P]),
+    "pa_sched_last_swaps": (c_int32, [_P, _I64P, c_int32, _I32P, _I64P, c_int32, _I32P]),
     "pa_sched_request_info": (c_int32, [_P, c_int64, POINTER(RequestInfo)]),
     "pa_sched_stats": (c_int32, [_P, POINTER(SchedStats)]),
     "pa_reshape_and_cache": (c_int32, [_P, _P, _P, _P, _P, c_int32, c_int32, c_int32, c_int32, c_int32, _P, _P]),

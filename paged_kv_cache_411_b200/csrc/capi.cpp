@@ -28,7 +28,7 @@ pa_status cuda_status(cudaError_t e, const char* where, const char* why) {
 
 extern "C" {
 
-int32_t pa_abi_version(void) { return 1; }
+int32_t pa_abi_version(void) { return 2; }
 
 const char* pa_last_error(void) { return pagedkv::last_error(); }
 

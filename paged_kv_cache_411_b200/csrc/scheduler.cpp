@@ -19,6 +19,18 @@
 //      a chunk of at most the remaining token budget (max_num_tokens); without
 //      chunked prefill a prompt runs only whole.  A chunk that cannot get its
 //      blocks waits for a later step.
+// With a CPU pool attached (pa_sched_enable_swap), step 2 preempts by the
+// page's second strategy instead (§5.4 "Swap to CPU" with §4.4's swap_out):
+// the victim's blocks move to the CPU pool (pa_alloc_swap_out bookkeeping:
+// CPU blocks allocated first, block i to block i, GPU blocks freed) and it
+// waits, progress kept, in a swapped queue (most recently preempted first);
+// a victim the CPU pool cannot take is recomputed.  Before admission,
+// swapped requests come back in queue order while seats are free and the
+// blocks of their table (plus one if their next decode opens a block), the
+// decodes' needs and the watermark are available; no waiting request is
+// admitted while one is still swapped.  The step reports the block moves
+// (pa_sched_last_swaps), which the caller performs, swap-outs first, before
+// the step's kernels.
 // The step's slot mapping lists the prefill rows (in prefill order) and then
 // the decode rows.  pa_sched_complete then applies the step: chunks become
 // cached, a request whose prefill completed emits a token, each decode emits
@@ -35,7 +47,7 @@ using pagedkv::fail;
 
 namespace {
 
-enum : int32_t { kWaiting = 0, kRunning = 1, kFinished = 2 };
+enum : int32_t { kWaiting = 0, kRunning = 1, kFinished = 2, kSwapped = 3 };
 
 struct Req {
     int32_t prompt_len = 0;
@@ -58,6 +70,10 @@ struct Entry {
 
 struct pa_sched {
     pa_alloc* alloc = nullptr;
+    pa_alloc* cpu = nullptr;       // CPU pool for swap preemption (NULL: recompute)
+    std::deque<int64_t> swapped;   // front = most recently preempted
+    std::vector<int64_t> swap_out_pairs, swap_in_pairs;   // (src, dst) block pairs of the last step
+    int64_t swap_outs = 0, swap_ins = 0;
     pa_sched_config_t cfg{};
     int32_t block_size = 0;
     std::unordered_map<int64_t, Req> reqs;
@@ -78,6 +94,15 @@ struct pa_sched {
         return n;
     }
     bool decoding(const Req& q) const { return q.state == kRunning && q.prefilled == q.to_prefill && q.generated < q.max_new; }
+    // the block table of r in allocator a (both pools hold ceil(seq_len / block_size) blocks)
+    std::vector<int32_t> table(const pa_alloc* a, int64_t r) const {
+        int32_t len = 0, n = 0;
+        if (pa_alloc_seq_len(a, r, &len) != PA_OK) return {};
+        std::vector<int32_t> t((len + block_size - 1) / block_size);
+        if (pa_alloc_get_block_table(a, r, t.data(), static_cast<int32_t>(t.size()), &n) != PA_OK) return {};
+        t.resize(n);
+        return t;
+    }
 };
 
 extern "C" {
@@ -99,6 +124,38 @@ pa_status pa_sched_create(pa_alloc* alloc, const pa_sched_config_t* cfg, pa_sche
 }
 
 void pa_sched_destroy(pa_sched* s) { delete s; }
+
+pa_status pa_sched_enable_swap(pa_sched* s, pa_alloc* cpu) {
+    if (!s) return fail(PA_ERR_INVALID_ARG, "pa_sched_enable_swap: NULL scheduler");
+    if (s->step_open) return fail(PA_ERR_INVALID_ARG, "pa_sched_enable_swap: a step is open");
+    if (!cpu) {
+        if (!s->swapped.empty())
+            return fail(PA_ERR_INVALID_ARG, "pa_sched_enable_swap: requests are still swapped out");
+        s->cpu = nullptr;
+        return PA_OK;
+    }
+    pa_alloc_stats_t st;
+    pa_alloc_stats(cpu, &st);
+    if (st.block_size != s->block_size)
+        return fail(PA_ERR_INVALID_ARG, "pa_sched_enable_swap: CPU pool block size %d differs from %d",
+                    st.block_size, s->block_size);
+    s->cpu = cpu;
+    return PA_OK;
+}
+
+pa_status pa_sched_last_swaps(const pa_sched* s, int64_t* out_pairs, int32_t out_cap, int32_t* n_out,
+                              int64_t* in_pairs, int32_t in_cap, int32_t* n_in) {
+    if (!s) return fail(PA_ERR_INVALID_ARG, "pa_sched_last_swaps: NULL scheduler");
+    const int32_t no = static_cast<int32_t>(s->swap_out_pairs.size() / 2);
+    const int32_t ni = static_cast<int32_t>(s->swap_in_pairs.size() / 2);
+    if (n_out) *n_out = no;
+    if (n_in) *n_in = ni;
+    if ((out_pairs && out_cap < no) || (in_pairs && in_cap < ni))
+        return fail(PA_ERR_INVALID_ARG, "pa_sched_last_swaps: capacity below %d / %d pairs", no, ni);
+    for (size_t i = 0; out_pairs && i < s->swap_out_pairs.size(); ++i) out_pairs[i] = s->swap_out_pairs[i];
+    for (size_t i = 0; in_pairs && i < s->swap_in_pairs.size(); ++i) in_pairs[i] = s->swap_in_pairs[i];
+    return PA_OK;
+}
 
 pa_status pa_sched_add_request(pa_sched* s, int64_t req, int32_t prompt_len, int32_t max_new_tokens) {
     if (!s || prompt_len <= 0 || max_new_tokens <= 0)
@@ -123,6 +180,8 @@ pa_status pa_sched_step(pa_sched* s, pa_step_info_t* info, int64_t* prefill_reqs
     if (s->step_open) return fail(PA_ERR_INVALID_ARG, "pa_sched_step: the previous step was not completed");
     pa_step_info_t inf{};
     const int32_t bs = s->block_size;
+    s->swap_out_pairs.clear();
+    s->swap_in_pairs.clear();
     // 1. free the requests that produced their last token
     std::vector<int64_t> keep;
     for (int64_t r : s->running) {
@@ -147,17 +206,56 @@ pa_status pa_sched_step(pa_sched* s, pa_step_info_t* info, int64_t* prefill_reqs
         const int64_t v = s->running.back();
         s->running.pop_back();
         Req& q = s->reqs[v];
+        q.preemptions += 1;
+        inf.num_preempted += 1;
+        if (s->cpu) {
+            const std::vector<int32_t> gt = s->table(s->alloc, v);
+            if (pa_alloc_swap_out(s->alloc, s->cpu, v, nullptr, nullptr, nullptr, nullptr, 0, nullptr) == PA_OK) {
+                const std::vector<int32_t> ct = s->table(s->cpu, v);
+                for (size_t i = 0; i < gt.size(); ++i) {
+                    s->swap_out_pairs.push_back(gt[i]);
+                    s->swap_out_pairs.push_back(ct[i]);
+                }
+                q.state = kSwapped;
+                s->swapped.push_front(v);
+                s->swap_outs += 1;
+                need = decode_need();
+                continue;
+            }
+        }
         pa_alloc_free(s->alloc, v);
         q.to_prefill = q.prompt_len + q.generated;
         q.prefilled = 0;
         q.state = kWaiting;
-        q.preemptions += 1;
         s->waiting.push_front(v);
-        inf.num_preempted += 1;
         need = decode_need();
     }
-    // 3. admit in arrival order while the prefill's blocks fit beside the decodes and the watermark
-    while (static_cast<int32_t>(s->running.size()) < s->cfg.max_num_seqs && !s->waiting.empty()) {
+    // swapped requests come back first, while seats and blocks last
+    while (s->cpu && !s->swapped.empty() && static_cast<int32_t>(s->running.size()) < s->cfg.max_num_seqs) {
+        const int64_t r = s->swapped.front();
+        Req& q = s->reqs[r];
+        const std::vector<int32_t> ct = s->table(s->cpu, r);
+        int32_t len = 0;
+        pa_alloc_seq_len(s->cpu, r, &len);
+        const int64_t opens = (q.prefilled == q.to_prefill && q.generated < q.max_new && len % bs == 0) ? 1 : 0;
+        if (s->available() - need - s->cfg.watermark_blocks < static_cast<int64_t>(ct.size()) + opens) break;
+        s->swapped.pop_front();
+        pa_status st = pa_alloc_swap_in(s->alloc, s->cpu, r, nullptr, nullptr, nullptr, nullptr, 0, nullptr);
+        if (st != PA_OK) return st;
+        const std::vector<int32_t> gt = s->table(s->alloc, r);
+        for (size_t i = 0; i < ct.size(); ++i) {
+            s->swap_in_pairs.push_back(ct[i]);
+            s->swap_in_pairs.push_back(gt[i]);
+        }
+        q.state = kRunning;
+        s->running.push_back(r);
+        s->swap_ins += 1;
+        need += opens;
+    }
+    // 3. admit in arrival order while the prefill's blocks fit beside the decodes and the watermark (not
+    //    while a request is still swapped out)
+    while (s->swapped.empty() && static_cast<int32_t>(s->running.size()) < s->cfg.max_num_seqs &&
+           !s->waiting.empty()) {
         const int64_t r = s->waiting.front();
         Req& q = s->reqs[r];
         const int64_t blocks = (static_cast<int64_t>(q.to_prefill) + bs - 1) / bs;
@@ -276,6 +374,9 @@ pa_status pa_sched_stats(const pa_sched* s, pa_sched_stats_t* out) {
     for (const auto& kv : s->reqs) out->preemptions += kv.second.preemptions;
     out->prefill_tokens = s->prefill_tokens;
     out->decode_tokens = s->decode_tokens;
+    out->swapped = static_cast<int64_t>(s->swapped.size());
+    out->swap_outs = s->swap_outs;
+    out->swap_ins = s->swap_ins;
     return PA_OK;
 }
 

@@ -33,7 +33,7 @@ def test_library_exports_every_declared_symbol():
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(_lib.SIGNATURES), "ctypes signatures out of sync with the header"
-    assert lib.pa_abi_version() == 1
+    assert lib.pa_abi_version() == 2
 
 
 def test_status_strings_and_device_flag():
@@ -234,3 +234,34 @@ def test_stall_hook_arguments():
     assert lib.pa_debug_inject_stall(3, 1000) == pk.PA_ERR_INVALID_ARG
     assert lib.pa_debug_inject_stall(pk.PA_KERNEL_DECODE, 0) == pk.PA_ERR_INVALID_ARG
     assert lib.pa_debug_inject_stall(pk.PA_KERNEL_PREFILL, 3_000_000_000) == pk.PA_ERR_INVALID_ARG
+
+
+def test_pack_into_caller_arrays_matches_allocating_path():
+    """pack(tables=, lens=) writes into the caller's (e.g. pinned staging) arrays exactly what the
+    allocating form returns, -1 padding included; wrong dtypes, shapes, layouts and read-only views
+    are refused before the C call can write through them."""
+    a = pk.BlockAllocator(32, 4)
+    for r, n in ((1, 9), (2, 1), (3, 16), (4, 0)):
+        assert a.allocate(r, n) == pk.PA_OK
+    reqs = [3, 1, 4, 2]
+    st, t0, l0 = a.pack(reqs, 6)
+    assert st == pk.PA_OK
+    buf = np.full(4 * 6 + 4 + 3, 12345, dtype=np.int32)
+    tv, lv = buf[:24].reshape(4, 6), buf[24:28]
+    st, t1, l1 = a.pack(reqs, 6, tables=tv, lens=lv)
+    assert st == pk.PA_OK and t1 is tv and l1 is lv
+    assert np.array_equal(tv, t0) and np.array_equal(lv, l0)
+    assert (tv[2] == -1).all() and tv[1, 3:].tolist() == [-1, -1, -1]
+    assert buf[28:].tolist() == [12345] * 3                       # nothing written past the views
+    with pytest.raises(ValueError):
+        a.pack(reqs, 6, tables=np.zeros((4, 6), np.int64))
+    with pytest.raises(ValueError):
+        a.pack(reqs, 6, tables=np.zeros((4, 5), np.int32))
+    with pytest.raises(ValueError):
+        a.pack(reqs, 6, tables=np.zeros((6, 4), np.int32).T)
+    with pytest.raises(ValueError):
+        a.pack(reqs, 6, lens=np.broadcast_to(np.zeros(1, np.int32), (4,)))
+    ro = np.zeros((4, 6), np.int32)
+    ro.flags.writeable = False
+    with pytest.raises(ValueError):
+        a.pack(reqs, 6, tables=ro)

@@ -32,8 +32,9 @@ def run_oracle_scheduler_trace(case):
     """Replays one golden case through the oracle scheduler and checks every step and the end state."""
     cfg = case["config"]
     bm = PrefixCachingBlockManager(cfg["num_blocks"], cfg["block_size"])
+    cpu = obm.BlockManager(cfg["swap_cpu_blocks"], cfg["block_size"]) if "swap_cpu_blocks" in cfg else None
     sched = osch.Scheduler(bm, cfg["max_num_seqs"], cfg["max_num_tokens"], cfg["chunked_prefill"],
-                           cfg["watermark_blocks"])
+                           cfg["watermark_blocks"], swap_cpu=cpu)
     for i, want in enumerate(case["steps"]):
         for r in case["requests"]:
             if r["arrival"] == i:
@@ -45,9 +46,14 @@ def run_oracle_scheduler_trace(case):
         assert [list(p) for p in got["prefill"]] == want["prefill"], (case["name"], i, "prefill")
         assert [list(d) for d in got["decode"]] == want["decode"], (case["name"], i, "decode")
         assert got["slot_mapping"] == want["slot_mapping"], (case["name"], i, "slots")
+        if "swap_out" in want:
+            assert [list(x) for x in got["swap_out"]] == want["swap_out"], (case["name"], i, "swap_out")
+            assert [list(x) for x in got["swap_in"]] == want["swap_in"], (case["name"], i, "swap_in")
         sched.complete()
     fin = case["final"]
     assert bm.free_blocks == fin["free_list"]
+    if cpu is not None:
+        assert cpu.free_blocks == fin["cpu_free_list"]
     assert {str(r): t for r, t in bm.block_tables.items()} == fin["tables"]
     for rid, want in fin["requests"].items():
         q = sched.reqs[int(rid)]
@@ -68,6 +74,10 @@ def test_cpp_scheduler_follows_hand_trace(name):
     alloc = pk.BlockAllocator(cfg["num_blocks"], cfg["block_size"])
     sched = pk.Scheduler(alloc, max_num_seqs=cfg["max_num_seqs"], max_num_tokens=cfg["max_num_tokens"],
                          chunked_prefill=cfg["chunked_prefill"], watermark_blocks=cfg["watermark_blocks"])
+    cpu = None
+    if "swap_cpu_blocks" in cfg:
+        cpu = pk.BlockAllocator(cfg["swap_cpu_blocks"], cfg["block_size"])
+        assert sched.enable_swap(cpu) == pk.PA_OK
     for i, want in enumerate(case["steps"]):
         for r in case["requests"]:
             if r["arrival"] == i:
@@ -79,9 +89,13 @@ def test_cpp_scheduler_follows_hand_trace(name):
                 zip(got["prefill_reqs"], got["prefill_ctx"], got["prefill_len"])] == want["prefill"], (name, i)
         assert [[int(a), int(b)] for a, b in zip(got["decode_reqs"], got["decode_seq_lens"])] == want["decode"]
         assert got["slot_mapping"].tolist() == want["slot_mapping"], (name, i)
+        if "swap_out" in want:
+            assert got["swap_out"].tolist() == want["swap_out"] and got["swap_in"].tolist() == want["swap_in"], (name, i)
         sched.complete()
     fin = case["final"]
     assert alloc.free_list().tolist() == fin["free_list"]
+    if cpu is not None:
+        assert cpu.free_list().tolist() == fin["cpu_free_list"]
     for rid, t in fin["tables"].items():
         assert alloc.get_block_table(int(rid))[1].tolist() == t
     for rid, want in fin["requests"].items():

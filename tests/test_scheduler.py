@@ -11,18 +11,23 @@ from oracle import scheduler as osch
 from oracle.prefix_cache import PrefixCachingBlockManager
 
 
-def _pair(N, bs, **cfg):
+def _pair(N, bs, cpu_blocks=None, **cfg):
     ca = pk.BlockAllocator(N, bs)
     cs = pk.Scheduler(ca, **cfg)
     om = PrefixCachingBlockManager(N, bs)
+    ocpu = None
+    if cpu_blocks is not None:
+        cs._keep_cpu = pk.BlockAllocator(cpu_blocks, bs)
+        assert cs.enable_swap(cs._keep_cpu) == pk.PA_OK
+        ocpu = obm.BlockManager(cpu_blocks, bs)
     os_ = osch.Scheduler(om, cfg["max_num_seqs"], cfg["max_num_tokens"], cfg.get("chunked_prefill", True),
-                         cfg.get("watermark_blocks", 0))
+                         cfg.get("watermark_blocks", 0), swap_cpu=ocpu)
     return ca, cs, om, os_
 
 
-def _run(trace, N, bs, steps, **cfg):
+def _run(trace, N, bs, steps, cpu_blocks=None, **cfg):
     """trace: [(arrival_step, prompt_len, max_new)], request ids = index."""
-    ca, cs, om, os_ = _pair(N, bs, **cfg)
+    ca, cs, om, os_ = _pair(N, bs, cpu_blocks, **cfg)
     pending = sorted(range(len(trace)), key=lambda i: trace[i][0])
     k = 0
     log = []
@@ -40,6 +45,9 @@ def _run(trace, N, bs, steps, **cfg):
             == b["prefill"]
         assert [(int(r), int(n)) for r, n in zip(a["decode_reqs"], a["decode_seq_lens"])] == b["decode"]
         assert a["slot_mapping"].tolist() == b["slot_mapping"]
+        if cpu_blocks is not None:
+            assert a["swap_out"].tolist() == [list(x) for x in b["swap_out"]], step
+            assert a["swap_in"].tolist() == [list(x) for x in b["swap_in"]], step
         cs.complete()
         os_.complete()
         log.append(a)
@@ -63,6 +71,26 @@ trace_st = st.lists(st.tuples(st.integers(0, 12), st.integers(1, 90), st.integer
 def test_cpp_scheduler_matches_oracle(trace, N, bs, max_seqs, max_tokens, chunked, watermark):
     _run(trace, N, bs, 40, max_num_seqs=max_seqs, max_num_tokens=max_tokens, chunked_prefill=chunked,
          watermark_blocks=watermark)
+
+
+@settings(max_examples=200, deadline=None)
+@given(trace_st, st.integers(4, 40), st.integers(0, 30), st.sampled_from([1, 4, 16]), st.integers(1, 6),
+       st.integers(1, 64), st.booleans(), st.integers(0, 2))
+def test_cpp_swap_scheduler_matches_oracle(trace, N, ncpu, bs, max_seqs, max_tokens, chunked, watermark):
+    """Swap preemption ([CB-PA] §5.4 strategy 2): plans, block moves and end states agree, including CPU
+    pools too small to take a victim (recompute fallback)."""
+    _run(trace, N, bs, 40, cpu_blocks=ncpu, max_num_seqs=max_seqs, max_num_tokens=max_tokens,
+         chunked_prefill=chunked, watermark_blocks=watermark)
+
+
+def test_swap_preemption_keeps_progress():
+    """A pool too small for two long generations, with a CPU pool: the newer request is swapped out and
+    back instead of recomputed, every request finishes, and nothing stays on the CPU."""
+    cs, os_, log = _run([(0, 16, 40), (0, 16, 40)], 10, 8, 200, cpu_blocks=8, max_num_seqs=2, max_num_tokens=64)
+    st = cs.stats()
+    assert st["swap_outs"] >= 1 and st["swap_ins"] == st["swap_outs"] and st["swapped"] == 0
+    assert os_.reqs[1].to_prefill == 16 and os_.reqs[1].preemptions >= 1     # nothing recomputed
+    assert cs._keep_cpu.stats()["num_free"] == 8
 
 
 def test_seeded_trace_serves_everything():

@@ -1,7 +1,8 @@
 """The continuous-batching step driver running the kernels (GPU).
 
 The C++ scheduler plans every step of a seeded arrival trace (mixed prefill
-chunks and decodes, preemption by recomputation under a small pool); each
+chunks and decodes, preemption by recomputation -- or by swapping to a host
+pool -- under a small pool); each
 step writes its rows with reshape_and_cache and runs the prefill and decode
 kernels on the planned tables.  Every output row is checked against the
 float64 oracle's attention over the request's logical K/V (a recomputed
@@ -18,6 +19,18 @@ TOL = 2e-3
 
 
 def test_scheduler_drives_kernels(cuda_ready):
+    _serve(swap=False)
+
+
+def test_scheduler_with_swap_preemption_drives_kernels(cuda_ready):
+    """[CB-PA] §5.4 strategy 2: preempted requests move to a pinned host pool and back.  Each step the
+    block moves the scheduler reports run first (GPU to host, then host to GPU, pa_swap_blocks on the
+    stream), then the step's kernels.  A swapped-in request's blocks hold its K/V bit for bit, it is
+    never recomputed, and every output row matches the oracle."""
+    _serve(swap=True)
+
+
+def _serve(swap):
     H, D, bs, N = 4, 128, 16, 14            # a pool that forces preemptions
     scale = 1 / np.sqrt(D)
     rng = np.random.default_rng(30)
@@ -32,6 +45,14 @@ def test_scheduler_drives_kernels(cuda_ready):
     sched = pk.Scheduler(alloc, max_num_seqs=6, max_num_tokens=64)
     kc = torch.full((N, bs, H, D), float("nan"), dtype=torch.float16, device="cuda")
     vc = torch.full_like(kc, float("nan"))
+    NC = 40
+    block_bytes = bs * H * D * 2
+    if swap:
+        cpu = pk.BlockAllocator(NC, bs)
+        assert sched.enable_swap(cpu) == pk.PA_OK
+        ck = torch.full((NC, bs, H, D), float("nan"), dtype=torch.float16).pin_memory()
+        cv = torch.full_like(ck, float("nan")).pin_memory()
+    swapped_in = 0
     mb = -(-maxlen // bs)
     ws = torch.empty(pk.decode_workspace_bytes(6, H, D, mb, bs), dtype=torch.uint8, device="cuda")
     added, checked_rows, preempted, mixed = 0, 0, 0, 0
@@ -41,6 +62,26 @@ def test_scheduler_drives_kernels(cuda_ready):
             added += 1
         plan = sched.step()
         preempted += plan["num_preempted"]
+        if swap:
+            if len(plan["swap_out"]):
+                pk.swap_blocks(kc, vc, ck, cv, plan["swap_out"], block_bytes, N, NC)
+            if len(plan["swap_in"]):
+                pk.swap_blocks(ck, cv, kc, vc, plan["swap_in"], block_bytes, NC, N)
+                torch.cuda.synchronize()
+                moved = {int(b) for b in plan["swap_in"][:, 1]}
+                for r in range(n):
+                    st, t = alloc.get_block_table(r)
+                    if st != pk.PA_OK or not moved & set(t.tolist()):
+                        continue
+                    # positions already cached: the step's own rows (a decode token, a chunk) come later
+                    n_kv = alloc.seq_len(r)[1] - int((plan["decode_reqs"] == r).sum()) \
+                        - int(plan["prefill_len"][plan["prefill_reqs"] == r].sum())
+                    idx = np.arange(n_kv)
+                    got_k = kc[torch.from_numpy(t[idx // bs]).cuda(), torch.from_numpy(idx % bs).cuda()]
+                    got_v = vc[torch.from_numpy(t[idx // bs]).cuda(), torch.from_numpy(idx % bs).cuda()]
+                    assert np.array_equal(got_k.cpu().numpy().view(np.int16), K[r][:n_kv].view(np.int16)), r
+                    assert np.array_equal(got_v.cpu().numpy().view(np.int16), V[r][:n_kv].view(np.int16)), r
+                    swapped_in += 1
         if plan["num_tokens"] == 0:
             sched.complete()
             if sched.stats()["finished"] == n:
@@ -95,3 +136,7 @@ def test_scheduler_drives_kernels(cuda_ready):
     for r in range(n):
         st, info = sched.request_info(r)
         assert info["generated"] == outs[r]
+    if swap:
+        assert stats["swap_outs"] > 0 and stats["swap_ins"] == stats["swap_outs"] and swapped_in > 0
+        assert stats["prefill_tokens"] == int(prompts.sum())      # nothing was recomputed
+        assert cpu.stats()["num_free"] == NC
