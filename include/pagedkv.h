@@ -205,7 +205,7 @@ typedef struct {
     int64_t evictable_blocks;  /* registered blocks with refcount 0 (the LRU)      */
     int64_t hit_blocks;        /* blocks reused by allocate_cached so far          */
     int64_t evictions;         /* parked blocks taken back for new content         */
-    int64_t prefix_nodes;      /* distinct block prefixes seen                     */
+    int64_t prefix_nodes;      /* block prefixes in the trie now                   */
 } pa_cache_stats_t;
 
 /* Allocate `req` for tokens[0..num_tokens) (host int32 token ids), reusing the
@@ -216,7 +216,33 @@ typedef struct {
  * Errors: EXISTS, OOM (nothing changes), INVALID_ARG. */
 pa_status pa_alloc_allocate_cached(pa_alloc* a, int64_t req, const int32_t* tokens, int32_t num_tokens,
                                    int32_t* cached_tokens_out);
-/* Prefix-cache counters. */
+/* The lookup pa_alloc_begin_cached makes, without taking anything: *hit_blocks
+ * (nullable) = cached blocks it would reuse for tokens[0..num_tokens), of
+ * which *parked_blocks (nullable) now sit in the LRU (a take would remove them
+ * from pa_alloc_available's count).  Errors: INVALID_ARG. */
+pa_status pa_alloc_cached_prefix(const pa_alloc* a, const int32_t* tokens, int32_t num_tokens,
+                                 int32_t* hit_blocks, int32_t* parked_blocks);
+/* Start `req` from the prefix cache ([CB-PA] §4.2 inside the §2.2 loop): its
+ * table becomes the cached blocks of the longest cached prefix of whole blocks
+ * of tokens[0..num_tokens), at most (num_tokens - 1) / block_size of them so
+ * that at least one token is left to compute (refcount + 1, taken out of the
+ * LRU), and seq_len = those blocks' tokens = *cached_tokens_out (nullable).
+ * Nothing new is taken: the caller appends the rest as it computes it.  The
+ * request is tracked: every block its appends fill, whose token ids are known
+ * (tokens, then pa_alloc_extend_tokens), is registered in the cache under the
+ * node of the block before it; tracking ends at the first filled block whose
+ * ids are unknown or whose content is already cached in another block.
+ * (pa_alloc_allocate_cached also tracks its request, when every full block it
+ * holds is its own node's block.)  Errors: EXISTS, INVALID_ARG. */
+pa_status pa_alloc_begin_cached(pa_alloc* a, int64_t req, const int32_t* tokens, int32_t num_tokens,
+                                int32_t* cached_tokens_out);
+/* Append the ids of tokens a tracked request generated to its known ids (a
+ * no-op for an untracked request).  Errors: NOT_FOUND, INVALID_ARG. */
+pa_status pa_alloc_extend_tokens(pa_alloc* a, int64_t req, const int32_t* ids, int32_t n);
+/* Prefix-cache counters.  A cache entry lives as long as its block: when an
+ * evicted block's prefix node has no children it is dropped, with every
+ * ancestor left without a block and without children, so prefix_nodes stays
+ * bounded by the cached blocks and their prefixes. */
 pa_status pa_alloc_cache_stats(const pa_alloc* a, pa_cache_stats_t* out);
 /* Copy the LRU of parked blocks, least recently parked first (the next
  * eviction takes out[0]).  Errors: INVALID_ARG (cap < length; *len_out set). */
@@ -308,6 +334,7 @@ typedef struct {
 
 typedef struct {
     int64_t steps, waiting, running, finished, preemptions, prefill_tokens, decode_tokens;
+    int64_t cached_tokens;      /* prompt tokens admission found in the prefix cache  */
     int64_t swapped;            /* requests swapped out now                           */
     int64_t swap_outs, swap_ins;  /* moves so far                                     */
 } pa_sched_stats_t;
@@ -319,6 +346,18 @@ void pa_sched_destroy(pa_sched* s);
  * (prompt_len or max_new_tokens <= 0), EXISTS (id known to the scheduler or
  * holding blocks in the allocator). */
 pa_status pa_sched_add_request(pa_sched* s, int64_t req, int32_t prompt_len, int32_t max_new_tokens);
+/* As pa_sched_add_request, with the prompt's token ids (host int32
+ * tokens[prompt_len], copied): the request goes through the allocator's
+ * prefix cache ([CB-PA] §4.2 in the §2.2 loop).  Admission looks up the
+ * longest cached prefix of the ids known so far (pa_alloc_cached_prefix),
+ * needs new blocks only for the rest, and starts the request from it
+ * (pa_alloc_begin_cached): those tokens are not prefilled again
+ * (pa_request_info_t.prefilled starts there).  The blocks its chunks and
+ * decodes fill become cacheable, and so do its generated tokens when their
+ * ids are reported with pa_sched_complete_tokens.  Errors: as
+ * pa_sched_add_request, INVALID_ARG (tokens NULL). */
+pa_status pa_sched_add_request_tokens(pa_sched* s, int64_t req, const int32_t* tokens, int32_t prompt_len,
+                                      int32_t max_new_tokens);
 /* Schedule one step (host buffers, any may be NULL): prefill_reqs /
  * prefill_ctx (tokens already cached) / prefill_len (chunk) and decode_reqs /
  * decode_seq_lens (including the new token) hold up to max_num_seqs entries;
@@ -334,6 +373,13 @@ pa_status pa_sched_step(pa_sched* s, pa_step_info_t* info, int64_t* prefill_reqs
  * that emitted max_new_tokens finishes (freed at the next step).
  * Errors: INVALID_ARG (no open step). */
 pa_status pa_sched_complete(pa_sched* s);
+/* pa_sched_complete, reporting the ids of the tokens the step emitted
+ * (host int32 ids[n], one per emitted token, in emission order: the requests
+ * whose prefill completed, in prefill order, then every decode); the ids of
+ * requests added with tokens extend their known ids.
+ * Errors: INVALID_ARG (no open step; n differs from the tokens emitted:
+ * nothing is applied). */
+pa_status pa_sched_complete_tokens(pa_sched* s, const int32_t* ids, int32_t n);
 
 /* Swap preemption ([CB-PA] §5.4 strategy 2 "Swap to CPU", §4.4 SwappingManager).
  * With a CPU-side allocator attached (same block_size; NULL detaches, allowed

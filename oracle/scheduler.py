@@ -38,6 +38,22 @@ where the page leaves the strategy open:
   available; no waiting request is admitted while a request is still swapped;
 * the step reports its block moves (GPU to CPU for the swap-outs, then CPU to
   GPU for the swap-ins), which the caller performs before the step's kernels.
+
+§4.2's automatic prefix caching inside the §2.2 loop, for requests whose token
+ids are given (``add_request(..., tokens=)``):
+
+* admission looks up the longest cached prefix of the ids it knows (prompt,
+  then generated tokens reported by ``complete(sampled=)``), needs new blocks
+  only for the rest (``blocks_needed(to_prefill) - hits``, with parked hits
+  no longer counted as available), and starts the request there
+  (``begin_cached``): the cached tokens are not prefilled again;
+* the blocks its prefill chunks and decodes fill are registered as they fill
+  (the allocator's tracked requests), and its generated ids are reported to
+  the allocator as they are emitted, so decoded text becomes cacheable too; a
+  request preempted by recomputation finds its own blocks in the cache when it
+  comes back;
+* ``complete(sampled)`` takes one id per emitted token, in emission order:
+  requests whose prefill completed (prefill order), then the decodes.
 """
 from __future__ import annotations
 
@@ -51,7 +67,8 @@ WAITING, RUNNING, FINISHED, SWAPPED = 0, 1, 2, 3
 
 
 class _Req:
-    def __init__(self, prompt_len, max_new):
+    def __init__(self, prompt_len, max_new, tokens=None):
+        self.tokens = None if tokens is None else [int(t) for t in tokens]
         self.prompt_len = prompt_len
         self.max_new = max_new
         self.to_prefill = prompt_len
@@ -79,11 +96,12 @@ class Scheduler:
         self.waiting: deque = deque()
         self.running: list = []
         self.steps = 0
+        self.cached_tokens = 0
         self.last_prefill: list = []
         self.last_decode: list = []
 
-    def add_request(self, req, prompt_len, max_new):
-        self.reqs[req] = _Req(prompt_len, max_new)
+    def add_request(self, req, prompt_len, max_new, tokens=None):
+        self.reqs[req] = _Req(prompt_len, max_new, tokens)
         self.waiting.append(req)
         return OK
 
@@ -174,12 +192,21 @@ class Scheduler:
         while len(self.running) < self.max_num_seqs and self.waiting:
             r = self.waiting[0]
             q = self.reqs[r]
-            if self.bm._available() - need - self.watermark < blocks_needed(q.to_prefill, bs):
+            hits, parked = 0, 0
+            if q.tokens is not None:
+                known = q.tokens[:q.to_prefill]
+                hits, parked = self.bm.cached_prefix(known)
+            if self.bm._available() - parked - need - self.watermark < blocks_needed(q.to_prefill, bs) - hits:
                 break
             self.waiting.popleft()
-            assert self.bm.allocate(r, 0) == OK
-            q.state = RUNNING
             q.prefilled = 0
+            if q.tokens is not None:
+                st, q.prefilled = self.bm.begin_cached(r, known)
+                self.cached_tokens += q.prefilled
+            else:
+                st = self.bm.allocate(r, 0)
+            assert st == OK
+            q.state = RUNNING
             self.running.append(r)
             info["num_admitted"] += 1
 
@@ -214,8 +241,17 @@ class Scheduler:
             budget -= chunk
         return slots
 
-    def complete(self):
+    def complete(self, sampled=None):
         now = self.steps
+        emitting = [r for r, ctx, chunk in self.last_prefill if self.reqs[r].prefilled + chunk == self.reqs[r].to_prefill]
+        emitting += [r for r, _ in self.last_decode]
+        if sampled is not None:
+            assert len(sampled) == len(emitting)
+            for r, t in zip(emitting, sampled):
+                q = self.reqs[r]
+                if q.tokens is not None:
+                    q.tokens.append(int(t))
+                    self.bm.extend_tokens(r, [int(t)])
 
         def emit(q):
             q.generated += 1

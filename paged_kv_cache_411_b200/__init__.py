@@ -149,6 +149,24 @@ class BlockAllocator:
         st = lib().pa_alloc_allocate_cached(self._h, req, _i32p(t), len(t), byref(n))
         return st, (n.value if st == PA_OK else 0)
 
+    def cached_prefix(self, tokens):
+        """(cached blocks begin_cached would reuse for tokens, of which parked in the LRU)."""
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        h, p = c_int32(0), c_int32(0)
+        check(lib().pa_alloc_cached_prefix(self._h, _i32p(t), len(t), byref(h), byref(p)))
+        return h.value, p.value
+
+    def begin_cached(self, req: int, tokens):
+        """Returns (status, cached_tokens): the request starts with its cached prefix only and is tracked."""
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        n = c_int32(0)
+        st = lib().pa_alloc_begin_cached(self._h, req, _i32p(t), len(t), byref(n))
+        return st, (n.value if st == PA_OK else 0)
+
+    def extend_tokens(self, req: int, ids) -> int:
+        t = np.ascontiguousarray(ids, dtype=np.int32)
+        return lib().pa_alloc_extend_tokens(self._h, req, _i32p(t), len(t))
+
     def cache_stats(self) -> dict:
         s = CacheStats()
         check(lib().pa_alloc_cache_stats(self._h, byref(s)))
@@ -193,8 +211,14 @@ class Scheduler:
         except Exception:
             pass
 
-    def add_request(self, req: int, prompt_len: int, max_new_tokens: int) -> int:
-        return lib().pa_sched_add_request(self._h, req, prompt_len, max_new_tokens)
+    def add_request(self, req: int, prompt_len: int, max_new_tokens: int, tokens=None) -> int:
+        """Queue a request; with its prompt's token ids it goes through the prefix cache."""
+        if tokens is None:
+            return lib().pa_sched_add_request(self._h, req, prompt_len, max_new_tokens)
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        if len(t) != prompt_len:
+            raise ValueError("add_request: len(tokens) must equal prompt_len")
+        return lib().pa_sched_add_request_tokens(self._h, req, _i32p(t), prompt_len, max_new_tokens)
 
     def step(self) -> dict:
         """Schedule one step; returns info plus the prefill/decode entries and the slot mapping."""
@@ -226,8 +250,13 @@ class Scheduler:
         check(lib().pa_sched_last_swaps(self._h, _i64p(out), no.value, byref(no), _i64p(inn), ni.value, byref(ni)))
         return out, inn
 
-    def complete(self) -> None:
-        check(lib().pa_sched_complete(self._h))
+    def complete(self, sampled=None) -> None:
+        """Apply the step; `sampled` (optional) = the ids of the tokens it emitted, in emission order."""
+        if sampled is None:
+            check(lib().pa_sched_complete(self._h))
+            return
+        t = np.ascontiguousarray(sampled, dtype=np.int32)
+        check(lib().pa_sched_complete_tokens(self._h, _i32p(t), len(t)))
 
     def request_info(self, req: int):
         from ._lib import RequestInfo

@@ -87,7 +87,8 @@ class RequestInfo(ctypes.Structure):
 
 class SchedStats(ctypes.Structure):
     _fields_ = [(k, c_int64) for k in ("steps", "waiting", "running", "finished", "preemptions",
-                                        "prefill_tokens", "decode_tokens", "swapped", "swap_outs", "swap_ins")]
+                                        "prefill_tokens", "decode_tokens", "cached_tokens", "swapped", "swap_outs",
+                                        "swap_ins")]
 
     def as_dict(self):
         return {k: getattr(self, k) for k, _ in self._fields_}
@@ -121,6 +122,9 @@ SIGNATURES = {
     "pa_alloc_free_list": (c_int32, [_P, _I32P, c_int32, _I32P]),
     "pa_alloc_allocate_cached": (c_int32, [_P, c_int64, _I32P, c_int32, _I32P]),
     "pa_alloc_cache_stats": (c_int32, [_P, POINTER(CacheStats)]),
+    "pa_alloc_cached_prefix": (c_int32, [_P, _I32P, c_int32, _I32P, _I32P]),
+    "pa_alloc_begin_cached": (c_int32, [_P, c_int64, _I32P, c_int32, _I32P]),
+    "pa_alloc_extend_tokens": (c_int32, [_P, c_int64, _I32P, c_int32]),
     "pa_alloc_evictable_list": (c_int32, [_P, _I32P, c_int32, _I32P]),
     "pa_swap_blocks": (c_int32, [_P, _P, _P, _P, _I64P, c_int32, c_int64, c_int32, c_int32, _P]),
     "pa_alloc_swap_out": (c_int32, [_P, _P, c_int64, _P, _P, _P, _P, c_int64, _P]),
@@ -130,6 +134,8 @@ SIGNATURES = {
     "pa_sched_add_request": (c_int32, [_P, c_int64, c_int32, c_int32]),
     "pa_sched_step": (c_int32, [_P, POINTER(StepInfo), _I64P, _I32P, _I32P, _I64P, _I32P, _I64P]),
     "pa_sched_complete": (c_int32, [_P]),
+    "pa_sched_complete_tokens": (c_int32, [_P, _I32P, c_int32]),
+    "pa_sched_add_request_tokens": (c_int32, [_P, c_int64, _I32P, c_int32, c_int32]),
     "pa_sched_enable_swap": (c_int32, [_P, _P]),
     "pa_sched_last_swaps": (c_int32, [_P, _I64P, c_int32, _I32P, _I64P, c_int32, _I32P]),
     "pa_sched_request_info": (c_int32, [_P, c_int64, POINTER(RequestInfo)]),

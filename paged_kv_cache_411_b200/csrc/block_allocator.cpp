@@ -27,7 +27,17 @@
 //     in an LRU of evictable blocks (a request's blocks are parked last block
 //     first, so a prefix is always at least as recent as its extensions);
 //   * a take pops the free list, or, when it is empty, evicts the least
-//     recently used parked block (its cache entry is dropped).
+//     recently used parked block (its cache entry is dropped);
+//   * a cache entry lives as long as its block: when an evicted block's node
+//     has no children it is dropped, and so, walking up, is every ancestor
+//     left without a block and without children (node ids are never reused),
+//     so the trie stays bounded by the blocks it describes;
+//   * begin_cached starts a request with only the cached blocks of the
+//     longest cached prefix that leaves at least one token to compute, and a
+//     request started by begin_cached or allocate_cached is tracked: its known
+//     token ids (extend_tokens adds generated ones) register every block its
+//     appends fill, under the node of the block before it, until a filled
+//     block's ids are unknown or its content is already cached elsewhere.
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
@@ -85,6 +95,9 @@ struct pa_alloc {
     struct Request {
         std::vector<int32_t> table;
         int32_t len = 0;
+        bool tracked = false;               // its filled blocks get registered
+        std::vector<int32_t> tokens;        // known token ids (tracked requests)
+        int64_t last_node = -1;             // node of its last registered block (-1: the root)
     };
     int32_t num_blocks = 0;
     int32_t block_size = 0;
@@ -94,6 +107,9 @@ struct pa_alloc {
     int64_t oom_count = 0;
     // prefix cache
     std::unordered_map<PrefixKey, int64_t, PrefixKeyHash> trie;   // (parent node, tokens) -> node
+    std::unordered_map<int64_t, PrefixKey> node_key;               // node -> its key
+    std::unordered_map<int64_t, int32_t> children;                 // node -> child nodes
+    int64_t next_node = 0;
     std::unordered_map<int64_t, int32_t> cache;                    // node -> block
     std::vector<int64_t> block_node;                               // block -> node, -1 if not registered
     std::list<int32_t> lru;                                        // parked blocks, least recent first
@@ -115,12 +131,26 @@ struct pa_alloc {
         } else {
             b = lru.front();
             unpark(b);
-            cache.erase(block_node[b]);
+            const int64_t node = block_node[b];
+            cache.erase(node);
             block_node[b] = -1;
             evictions += 1;
+            prune(node);
         }
         refcount[b] += 1;
         return b;
+    }
+    // Drops `node`, then its ancestors, while they hold no block and have no children.
+    void prune(int64_t node) {
+        while (node >= 0 && !cache.count(node) && children[node] == 0) {
+            auto k = node_key.find(node);
+            const int64_t parent = k->second.parent;
+            trie.erase(k->second);
+            node_key.erase(k);
+            children.erase(node);
+            node = parent;
+            if (node >= 0) children[node] -= 1;
+        }
     }
     // Drop one reference to every block of `table`; blocks reaching zero go to the free list
     // (unregistered, table order) or are parked in the LRU (registered, last block first).
@@ -143,9 +173,42 @@ struct pa_alloc {
         PrefixKey k{parent, std::vector<int32_t>(tokens, tokens + block_size)};
         auto it = trie.find(k);
         if (it != trie.end()) return it->second;
-        const int64_t node = static_cast<int64_t>(trie.size());
+        const int64_t node = next_node++;
+        node_key.emplace(node, k);
         trie.emplace(std::move(k), node);
+        children[node] = 0;
+        if (parent >= 0) children[parent] += 1;
         return node;
+    }
+    // Cached blocks (and their nodes) of the longest cached prefix of whole blocks, at most max_blocks.
+    void lookup_prefix(const int32_t* tokens, int64_t max_blocks, std::vector<int32_t>* hits,
+                       std::vector<int64_t>* nodes) const {
+        int64_t parent = -1;
+        for (int64_t i = 0; i < max_blocks; ++i) {
+            const int64_t node = lookup(parent, tokens + i * block_size);
+            if (node < 0) break;
+            auto c = cache.find(node);
+            if (c == cache.end()) break;
+            hits->push_back(c->second);
+            if (nodes) nodes->push_back(node);
+            parent = node;
+        }
+    }
+    // A tracked request just stored position len - 1: register its block if that filled it.
+    void on_append(Request& r) {
+        if (!r.tracked || r.len % block_size != 0) return;
+        if (static_cast<int64_t>(r.tokens.size()) < r.len) {
+            r.tracked = false;                       // ids unknown: the chain ends
+            return;
+        }
+        const int64_t node = intern(r.last_node, r.tokens.data() + (r.len - block_size));
+        if (cache.count(node)) {
+            r.tracked = false;                       // content cached in another block: the chain ends
+            return;
+        }
+        cache.emplace(node, r.table.back());
+        block_node[r.table.back()] = node;
+        r.last_node = node;
     }
     int64_t lookup(int64_t parent, const int32_t* tokens) const {
         PrefixKey k{parent, std::vector<int32_t>(tokens, tokens + block_size)};
@@ -226,6 +289,7 @@ pa_status pa_alloc_append_token(pa_alloc* a, int64_t req, int64_t* slot_out) {
     }
     if (slot_out) *slot_out = a->slot(r, r.len);
     r.len += 1;
+    a->on_append(r);
     return PA_OK;
 }
 
@@ -245,6 +309,7 @@ pa_status pa_alloc_append_tokens(pa_alloc* a, int64_t req, int32_t n, int64_t* s
         if (r.len % a->block_size == 0) r.table.push_back(a->take());
         if (slots_out) slots_out[i] = a->slot(r, r.len);
         r.len += 1;
+        a->on_append(r);
     }
     return PA_OK;
 }
@@ -378,15 +443,7 @@ pa_status pa_alloc_allocate_cached(pa_alloc* a, int64_t req, const int32_t* toke
     const int64_t nfull = num_tokens / bs, nblocks = a->blocks_for(num_tokens);
     // longest cached prefix of whole blocks
     std::vector<int32_t> hits;
-    int64_t parent = -1;
-    for (int64_t i = 0; i < nfull; ++i) {
-        const int64_t node = a->lookup(parent, tokens + i * bs);
-        if (node < 0) break;
-        auto c = a->cache.find(node);
-        if (c == a->cache.end()) break;
-        hits.push_back(c->second);
-        parent = node;
-    }
+    a->lookup_prefix(tokens, nfull, &hits, nullptr);
     int64_t parked_hits = 0;
     for (int32_t b : hits) parked_hits += a->in_lru[b] ? 1 : 0;
     const int64_t need = nblocks - static_cast<int64_t>(hits.size());
@@ -404,19 +461,72 @@ pa_status pa_alloc_allocate_cached(pa_alloc* a, int64_t req, const int32_t* toke
     }
     for (int64_t i = 0; i < need; ++i) r.table.push_back(a->take());
     // register the new full blocks under their prefix nodes
-    parent = -1;
+    int64_t parent = -1;
+    bool chain = true;
     for (int64_t i = 0; i < nfull; ++i) {
         const int64_t node = a->intern(parent, tokens + i * bs);
         if (i >= static_cast<int64_t>(hits.size()) && !a->cache.count(node)) {
             a->cache.emplace(node, r.table[i]);
             a->block_node[r.table[i]] = node;
         }
+        auto c = a->cache.find(node);
+        chain = chain && c != a->cache.end() && c->second == r.table[i];
         parent = node;
+    }
+    if (chain) {            // every full block is its own node's block: later filled blocks register too
+        r.tracked = true;
+        r.tokens.assign(tokens, tokens + num_tokens);
+        r.last_node = parent;
     }
     r.len = num_tokens;
     a->hit_blocks += static_cast<int64_t>(hits.size());
     a->reqs.emplace(req, std::move(r));
     if (cached_tokens_out) *cached_tokens_out = static_cast<int32_t>(hits.size()) * bs;
+    return PA_OK;
+}
+
+pa_status pa_alloc_cached_prefix(const pa_alloc* a, const int32_t* tokens, int32_t num_tokens, int32_t* hit_blocks,
+                                 int32_t* parked_blocks) {
+    if (!a || num_tokens < 0 || (num_tokens > 0 && !tokens))
+        return fail(PA_ERR_INVALID_ARG, "pa_alloc_cached_prefix: bad arguments");
+    std::vector<int32_t> hits;
+    a->lookup_prefix(tokens, num_tokens > 0 ? (num_tokens - 1) / a->block_size : 0, &hits, nullptr);
+    int32_t parked = 0;
+    for (int32_t b : hits) parked += a->in_lru[b] ? 1 : 0;
+    if (hit_blocks) *hit_blocks = static_cast<int32_t>(hits.size());
+    if (parked_blocks) *parked_blocks = parked;
+    return PA_OK;
+}
+
+pa_status pa_alloc_begin_cached(pa_alloc* a, int64_t req, const int32_t* tokens, int32_t num_tokens,
+                                int32_t* cached_tokens_out) {
+    if (!a || num_tokens < 0 || (num_tokens > 0 && !tokens))
+        return fail(PA_ERR_INVALID_ARG, "pa_alloc_begin_cached: bad arguments");
+    if (a->reqs.count(req)) return fail(PA_ERR_EXISTS, "pa_alloc_begin_cached: request %lld exists", (long long)req);
+    std::vector<int32_t> hits;
+    std::vector<int64_t> nodes;
+    a->lookup_prefix(tokens, num_tokens > 0 ? (num_tokens - 1) / a->block_size : 0, &hits, &nodes);
+    pa_alloc::Request r;
+    for (int32_t b : hits) {
+        if (a->in_lru[b]) a->unpark(b);
+        a->refcount[b] += 1;
+    }
+    r.table = hits;
+    r.len = static_cast<int32_t>(hits.size()) * a->block_size;
+    r.tracked = true;
+    r.tokens.assign(tokens, tokens + num_tokens);
+    r.last_node = nodes.empty() ? -1 : nodes.back();
+    a->hit_blocks += static_cast<int64_t>(hits.size());
+    a->reqs.emplace(req, std::move(r));
+    if (cached_tokens_out) *cached_tokens_out = static_cast<int32_t>(hits.size()) * a->block_size;
+    return PA_OK;
+}
+
+pa_status pa_alloc_extend_tokens(pa_alloc* a, int64_t req, const int32_t* ids, int32_t n) {
+    if (!a || n < 0 || (n > 0 && !ids)) return fail(PA_ERR_INVALID_ARG, "pa_alloc_extend_tokens: bad arguments");
+    auto it = a->reqs.find(req);
+    if (it == a->reqs.end()) return fail(PA_ERR_NOT_FOUND, "pa_alloc_extend_tokens: request %lld not found", (long long)req);
+    if (it->second.tracked) it->second.tokens.insert(it->second.tokens.end(), ids, ids + n);
     return PA_OK;
 }
 

@@ -31,10 +31,21 @@
 // admitted while one is still swapped.  The step reports the block moves
 // (pa_sched_last_swaps), which the caller performs, swap-outs first, before
 // the step's kernels.
+// Requests added with their token ids (pa_sched_add_request_tokens) use the
+// allocator's prefix cache (§4.2 inside the §2.2 loop): admission looks up
+// the longest cached prefix of the ids known so far (prompt, then the
+// generated ids pa_sched_complete_tokens reports), needs new blocks only for
+// the rest (parked hits no longer count as available) and starts the request
+// there with pa_alloc_begin_cached, so cached tokens are not prefilled again;
+// the blocks its chunks and decodes fill are registered as they fill, and the
+// generated ids go to the allocator as they are emitted, so decoded text
+// becomes cacheable and a request recomputed after preemption finds its own
+// blocks again.
 // The step's slot mapping lists the prefill rows (in prefill order) and then
 // the decode rows.  pa_sched_complete then applies the step: chunks become
 // cached, a request whose prefill completed emits a token, each decode emits
 // a token, and a request that has emitted max_new_tokens finishes.
+#include <algorithm>
 #include <cstdint>
 #include <deque>
 #include <new>
@@ -50,6 +61,8 @@ namespace {
 enum : int32_t { kWaiting = 0, kRunning = 1, kFinished = 2, kSwapped = 3 };
 
 struct Req {
+    bool has_tokens = false;
+    std::vector<int32_t> tokens;   // known ids: the prompt, then generated tokens as they are reported
     int32_t prompt_len = 0;
     int32_t max_new = 0;
     int32_t to_prefill = 0;        // tokens to prefill (prompt, plus generated tokens after a preemption)
@@ -81,7 +94,7 @@ struct pa_sched {
     std::vector<int64_t> running;  // admission order
     std::vector<Entry> last_prefill, last_decode;
     bool step_open = false;
-    int64_t steps = 0, preemptions = 0, finished = 0, prefill_tokens = 0, decode_tokens = 0;
+    int64_t steps = 0, preemptions = 0, finished = 0, prefill_tokens = 0, decode_tokens = 0, cached_tokens = 0;
 
     int64_t available() const {
         int64_t n = 0;
@@ -157,7 +170,21 @@ pa_status pa_sched_last_swaps(const pa_sched* s, int64_t* out_pairs, int32_t out
     return PA_OK;
 }
 
+static pa_status add_request(pa_sched* s, int64_t req, const int32_t* tokens, int32_t prompt_len,
+                             int32_t max_new_tokens);
+
 pa_status pa_sched_add_request(pa_sched* s, int64_t req, int32_t prompt_len, int32_t max_new_tokens) {
+    return add_request(s, req, nullptr, prompt_len, max_new_tokens);
+}
+
+pa_status pa_sched_add_request_tokens(pa_sched* s, int64_t req, const int32_t* tokens, int32_t prompt_len,
+                                      int32_t max_new_tokens) {
+    if (!tokens) return fail(PA_ERR_INVALID_ARG, "pa_sched_add_request_tokens: tokens is NULL");
+    return add_request(s, req, tokens, prompt_len, max_new_tokens);
+}
+
+static pa_status add_request(pa_sched* s, int64_t req, const int32_t* tokens, int32_t prompt_len,
+                             int32_t max_new_tokens) {
     if (!s || prompt_len <= 0 || max_new_tokens <= 0)
         return fail(PA_ERR_INVALID_ARG, "pa_sched_add_request: prompt_len and max_new_tokens must be positive");
     if (s->reqs.count(req)) return fail(PA_ERR_EXISTS, "pa_sched_add_request: request %lld exists", (long long)req);
@@ -165,6 +192,10 @@ pa_status pa_sched_add_request(pa_sched* s, int64_t req, int32_t prompt_len, int
     if (pa_alloc_seq_len(s->alloc, req, &dummy) == PA_OK)
         return fail(PA_ERR_EXISTS, "pa_sched_add_request: request %lld already holds blocks", (long long)req);
     Req r;
+    if (tokens) {
+        r.has_tokens = true;
+        r.tokens.assign(tokens, tokens + prompt_len);
+    }
     r.prompt_len = prompt_len;
     r.max_new = max_new_tokens;
     r.to_prefill = prompt_len;
@@ -258,13 +289,18 @@ pa_status pa_sched_step(pa_sched* s, pa_step_info_t* info, int64_t* prefill_reqs
            !s->waiting.empty()) {
         const int64_t r = s->waiting.front();
         Req& q = s->reqs[r];
-        const int64_t blocks = (static_cast<int64_t>(q.to_prefill) + bs - 1) / bs;
-        if (s->available() - need - s->cfg.watermark_blocks < blocks) break;
+        int32_t hits = 0, parked = 0;
+        const int32_t known = q.has_tokens ? std::min<int32_t>(static_cast<int32_t>(q.tokens.size()), q.to_prefill) : 0;
+        if (q.has_tokens) pa_alloc_cached_prefix(s->alloc, q.tokens.data(), known, &hits, &parked);
+        const int64_t blocks = (static_cast<int64_t>(q.to_prefill) + bs - 1) / bs - hits;
+        if (s->available() - parked - need - s->cfg.watermark_blocks < blocks) break;
         s->waiting.pop_front();
-        pa_status st = pa_alloc_allocate(s->alloc, r, 0);
-        if (st != PA_OK) return st;
-        q.state = kRunning;
         q.prefilled = 0;
+        pa_status st = q.has_tokens ? pa_alloc_begin_cached(s->alloc, r, q.tokens.data(), known, &q.prefilled)
+                                    : pa_alloc_allocate(s->alloc, r, 0);
+        if (st != PA_OK) return st;
+        s->cached_tokens += q.prefilled;
+        q.state = kRunning;
         s->running.push_back(r);
         inf.num_admitted += 1;
     }
@@ -320,8 +356,33 @@ pa_status pa_sched_step(pa_sched* s, pa_step_info_t* info, int64_t* prefill_reqs
     return PA_OK;
 }
 
-pa_status pa_sched_complete(pa_sched* s) {
+static pa_status complete_step(pa_sched* s, bool with_ids, const int32_t* ids, int32_t n);
+
+pa_status pa_sched_complete(pa_sched* s) { return complete_step(s, false, nullptr, 0); }
+
+pa_status pa_sched_complete_tokens(pa_sched* s, const int32_t* ids, int32_t n) {
+    if (n < 0 || (!ids && n > 0)) return fail(PA_ERR_INVALID_ARG, "pa_sched_complete_tokens: bad ids");
+    return complete_step(s, true, ids, n);
+}
+
+static pa_status complete_step(pa_sched* s, bool with_ids, const int32_t* ids, int32_t n) {
     if (!s || !s->step_open) return fail(PA_ERR_INVALID_ARG, "pa_sched_complete: no step to complete");
+    if (with_ids) {
+        // one id per emitted token: requests whose prefill completes (prefill order), then the decodes
+        std::vector<int64_t> emitting;
+        for (const Entry& e : s->last_prefill)
+            if (s->reqs[e.req].prefilled + e.b == s->reqs[e.req].to_prefill) emitting.push_back(e.req);
+        for (const Entry& e : s->last_decode) emitting.push_back(e.req);
+        if (static_cast<int32_t>(emitting.size()) != n)
+            return fail(PA_ERR_INVALID_ARG, "pa_sched_complete_tokens: %d ids for %zu emitted tokens", n,
+                        emitting.size());
+        for (int32_t i = 0; i < n; ++i) {
+            Req& q = s->reqs[emitting[i]];
+            if (!q.has_tokens) continue;
+            q.tokens.push_back(ids[i]);
+            pa_alloc_extend_tokens(s->alloc, emitting[i], ids + i, 1);
+        }
+    }
     const int64_t now = s->steps;
     auto emit = [&](Req& q) {
         q.generated += 1;
@@ -374,6 +435,7 @@ pa_status pa_sched_stats(const pa_sched* s, pa_sched_stats_t* out) {
     for (const auto& kv : s->reqs) out->preemptions += kv.second.preemptions;
     out->prefill_tokens = s->prefill_tokens;
     out->decode_tokens = s->decode_tokens;
+    out->cached_tokens = s->cached_tokens;
     out->swapped = static_cast<int64_t>(s->swapped.size());
     out->swap_outs = s->swap_outs;
     out->swap_ins = s->swap_ins;

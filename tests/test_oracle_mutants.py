@@ -298,6 +298,26 @@ class _RegisterPartialBlock(_PC):
         return st, cached
 
 
+class _NoPrune(_PC):
+    def _prune(self, node):
+        return None
+
+
+class _BeginTakesAll(_PC):
+    def _lookup(self, tokens, max_blocks):
+        return super()._lookup(tokens, len(tokens) // self.block_size)
+
+
+class _AppendsDoNotRegister(_PC):
+    def append_token(self, req):
+        return obm.BlockManager.append_token(self, req)
+
+
+class _PrefixIgnored(_Sched):
+    def add_request(self, req, prompt_len, max_new, tokens=None):
+        return super().add_request(req, prompt_len, max_new, None)
+
+
 def _floor_blocks(n, bs):
     return n // bs
 
@@ -367,7 +387,30 @@ MUTANTS = [
      [lambda: ppins.test_shared_system_prompt_is_stored_once()]),
     ("prefix cache registers the partial last block", opc, "PrefixCachingBlockManager", _RegisterPartialBlock,
      [lambda: ppins.test_oracle_follows_hand_trace()]),
+    ("prefix trie is never pruned", opc, "PrefixCachingBlockManager", _NoPrune,
+     [lambda: ppins.test_oracle_follows_tracked_hand_trace()]),
+    ("begin_cached reuses every full block", opc, "PrefixCachingBlockManager", _BeginTakesAll,
+     [lambda: ppins.test_oracle_follows_tracked_hand_trace()]),
+    ("filled blocks are not registered", opc, "PrefixCachingBlockManager", _AppendsDoNotRegister,
+     [lambda: ppins.test_oracle_follows_tracked_hand_trace()]),
+    ("scheduler ignores the prompt's token ids", osch, "Scheduler", _PrefixIgnored,
+     [lambda: _shared_prompt_pin()]),
 ]
+
+
+def _shared_prompt_pin():
+    """Oracle-only copy of the shared-prompt check: the second and third requests start at 32 cached tokens."""
+    system = list(range(100, 132))
+    prompts = [system + [1, 2, 3], system + [4, 5], system + [6] * 9]
+    sched = osch.Scheduler(opc.PrefixCachingBlockManager(64, 8), 4, 64)
+    ctx = []
+    for step in range(3):
+        sched.add_request(step, len(prompts[step]), 3, tokens=prompts[step])
+        info = sched.step()
+        ctx.append([c for _, c, _ in info["prefill"]])
+        sched.complete(sampled=[0] * (len(info["decode"]) + sum(
+            1 for r, c, n in info["prefill"] if sched.reqs[r].prefilled + n == sched.reqs[r].to_prefill)))
+    assert ctx == [[0], [32], [32]] and sched.cached_tokens == 64
 
 
 @pytest.mark.parametrize("name,module,attr,mutant,checks", MUTANTS, ids=[m[0] for m in MUTANTS])

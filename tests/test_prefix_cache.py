@@ -39,6 +39,69 @@ def test_oracle_follows_hand_trace():
             assert bm.refcount == op[1], op
 
 
+def _cached_prefixes(bm):
+    """Each cached block's whole token prefix (ids joined by commas) -> block."""
+    out = {}
+    for node, b in bm.cache.items():
+        toks, n = [], node
+        while n >= 0:
+            parent, blk = bm.node_key[n]
+            toks = list(blk) + toks
+            n = parent
+        out[",".join(map(str, toks))] = b
+    return out
+
+
+def run_tracked_trace(make):
+    """Replays the tracked-request golden through an allocator made by make(num_blocks, block_size); the
+    prefix-to-block checks need the oracle's trie, the rest runs on either side."""
+    g = golden("prefix_cache_tracked_trace.json")
+    bm = make(g["num_blocks"], g["block_size"])
+    ids = {"A": 1, "B": 2, "C": 3, "D": 4}
+    oracle = isinstance(bm, opc.PrefixCachingBlockManager)
+    names = (lambda x: x) if oracle else (lambda x: _NAMES[x])
+    for op in g["ops"]:
+        r = ids[op["req"]]
+        kind = op["op"]
+        if kind == "begin_cached":
+            st, cached = bm.begin_cached(r, op["tokens"])
+            assert (names(st), cached) == (op["status"], op["cached"]), op["why"]
+        elif kind == "append_tokens":
+            st, slots = bm.append_tokens(r, op["n"])
+            assert names(st) == op["status"] and list(slots) == op["slots"], op["why"]
+        elif kind == "append_token":
+            st, slot = bm.append_token(r)
+            assert names(st) == op["status"] and slot == op["slot"], op["why"]
+        elif kind == "extend_tokens":
+            assert names(bm.extend_tokens(r, op["ids"])) == op["status"]
+        elif kind == "allocate":
+            assert names(bm.allocate(r, op["tokens"])) == op["status"], op["why"]
+        else:
+            assert names(bm.free(r)) == op["status"]
+        tab = (lambda q: bm.block_tables[q]) if oracle else (lambda q: bm.get_block_table(q)[1].tolist())
+        if "table" in op:
+            assert tab(r) == op["table"], op["why"]
+        if "lru" in op:
+            assert (list(bm.lru) if oracle else bm.evictable_list().tolist()) == op["lru"], op["why"]
+        if "free" in op:
+            assert (bm.free_blocks if oracle else bm.free_list().tolist()) == op["free"], op["why"]
+        if "prefix_nodes" in op:
+            assert (len(bm.trie) if oracle else bm.cache_stats()["prefix_nodes"]) == op["prefix_nodes"], op["why"]
+        if "cached_prefixes" in op:
+            if oracle:
+                assert _cached_prefixes(bm) == op["cached_prefixes"], op["why"]
+            else:
+                assert bm.cache_stats()["cached_blocks"] == len(op["cached_prefixes"]), op["why"]
+
+
+def test_oracle_follows_tracked_hand_trace():
+    run_tracked_trace(opc.PrefixCachingBlockManager)
+
+
+def test_cpp_follows_tracked_hand_trace():
+    run_tracked_trace(pk.BlockAllocator)
+
+
 def test_shared_system_prompt_is_stored_once():
     """The page's figure: a 3-block system prompt shared by two requests with 2 private blocks
     each occupies 7 blocks; the second request finds all 3 prompt blocks in the cache."""
@@ -66,13 +129,23 @@ def test_shared_system_prompt_is_stored_once():
     assert bm.allocate_cached(6, system[bs:2 * bs] + [1]) == (obm.OK, 0)
 
 
+def _trie_is_pruned(om):
+    """Every prefix node holds a block or has a child (nothing dead is kept)."""
+    for node in om.node_key:
+        assert node in om.cache or om.children[node] > 0, node
+
+
+def _toks(fam, vocab, b, n):
+    base = [fam * 1000 + i for i in range(n)]
+    return base[: n - (b % 3)] + [(vocab * b + i) % 7 for i in range(b % 3)]
+
+
 def _replay(N, bs, log, vocab):
     ca = pk.BlockAllocator(N, bs)
     om = PrefixCachingBlockManager(N, bs)
     for kind, a, b, fam, n in log:
         if kind == 0:
-            base = [fam * 1000 + i for i in range(n)]
-            toks = base[: n - (b % 3)] + [(vocab * b + i) % 7 for i in range(b % 3)]
+            toks = _toks(fam, vocab, b, n)
             st, cached = ca.allocate_cached(a, toks)
             ost, ocached = om.allocate_cached(a, toks)
             assert (_NAMES[st], cached) == (ost, ocached)
@@ -85,10 +158,26 @@ def _replay(N, bs, log, vocab):
         elif kind == 3:
             p = min(n, om.seq_lens.get(a, 0))
             assert _NAMES[ca.fork(a, b, p)] == om.fork(a, b, p)
-        else:
+        elif kind == 4:
             assert _NAMES[ca.free(a)] == om.free(a)
+        elif kind == 5:
+            toks = _toks(fam, vocab, b, n)
+            assert ca.cached_prefix(toks) == om.cached_prefix(toks)
+            st, cached = ca.begin_cached(a, toks)
+            ost, ocached = om.begin_cached(a, toks)
+            assert (_NAMES[st], cached) == (ost, ocached)
+        elif kind == 6:
+            ids = [fam * 1000 + om.seq_lens.get(a, 0) + i for i in range(b + 1)]
+            assert _NAMES[ca.extend_tokens(a, ids)] == om.extend_tokens(a, ids)
+        else:
+            k = b % 4 + 1
+            st, slots = ca.append_tokens(a, k)
+            ost, oslots = om.append_tokens(a, k)
+            assert _NAMES[st] == ost and list(slots) == list(oslots)
         assert ca.free_list().tolist() == om.free_blocks
         assert ca.evictable_list().tolist() == list(om.lru)
+        assert ca.cache_stats()["prefix_nodes"] == len(om.trie)
+        _trie_is_pruned(om)
     for r in range(6):
         st, t = ca.get_block_table(r)
         assert t.tolist() == om.get_block_table(r)[1]
@@ -98,7 +187,7 @@ def _replay(N, bs, log, vocab):
     assert all(s1[k] == s2[k] for k in s2)
 
 
-ops = st.lists(st.tuples(st.integers(0, 4), st.integers(0, 5), st.integers(0, 5), st.integers(0, 2),
+ops = st.lists(st.tuples(st.integers(0, 7), st.integers(0, 5), st.integers(0, 5), st.integers(0, 2),
                          st.integers(0, 40)), min_size=1, max_size=120)
 
 

@@ -25,8 +25,14 @@ def _pair(N, bs, cpu_blocks=None, **cfg):
     return ca, cs, om, os_
 
 
-def _run(trace, N, bs, steps, cpu_blocks=None, **cfg):
-    """trace: [(arrival_step, prompt_len, max_new)], request ids = index."""
+def _sampled(r, k):
+    """The id a request emits as its k-th token (deterministic, from a small vocabulary)."""
+    return (r * 7919 + k * 31) % 11
+
+
+def _run(trace, N, bs, steps, cpu_blocks=None, prompts=None, **cfg):
+    """trace: [(arrival_step, prompt_len, max_new)], request ids = index; prompts: token ids per request
+    (prefix caching) or None."""
     ca, cs, om, os_ = _pair(N, bs, cpu_blocks, **cfg)
     pending = sorted(range(len(trace)), key=lambda i: trace[i][0])
     k = 0
@@ -34,8 +40,9 @@ def _run(trace, N, bs, steps, cpu_blocks=None, **cfg):
     for step in range(steps):
         while k < len(pending) and trace[pending[k]][0] <= step:
             i = pending[k]
-            assert cs.add_request(i, trace[i][1], trace[i][2]) == pk.PA_OK
-            os_.add_request(i, trace[i][1], trace[i][2])
+            toks = None if prompts is None else prompts[i]
+            assert cs.add_request(i, trace[i][1], trace[i][2], tokens=toks) == pk.PA_OK
+            os_.add_request(i, trace[i][1], trace[i][2], tokens=toks)
             k += 1
         a = cs.step()
         b = os_.step()
@@ -48,10 +55,20 @@ def _run(trace, N, bs, steps, cpu_blocks=None, **cfg):
         if cpu_blocks is not None:
             assert a["swap_out"].tolist() == [list(x) for x in b["swap_out"]], step
             assert a["swap_in"].tolist() == [list(x) for x in b["swap_in"]], step
-        cs.complete()
-        os_.complete()
+        if prompts is None:
+            cs.complete()
+            os_.complete()
+        else:
+            emit = [int(r) for r, c, n in b["prefill"] if os_.reqs[r].prefilled + n == os_.reqs[r].to_prefill]
+            emit += [int(r) for r, _ in b["decode"]]
+            ids = [_sampled(r, os_.reqs[r].generated) for r in emit]
+            cs.complete(sampled=ids)
+            os_.complete(sampled=ids)
+            assert ca.cache_stats()["prefix_nodes"] == len(om.trie)
+            assert ca.evictable_list().tolist() == list(om.lru)
         log.append(a)
     assert ca.free_list().tolist() == om.free_blocks
+    assert cs.stats()["cached_tokens"] == os_.cached_tokens
     for i in range(len(trace)):
         st_, info = cs.request_info(i)
         if st_ == pk.PA_OK:
@@ -81,6 +98,36 @@ def test_cpp_swap_scheduler_matches_oracle(trace, N, ncpu, bs, max_seqs, max_tok
     pools too small to take a victim (recompute fallback)."""
     _run(trace, N, bs, 40, cpu_blocks=ncpu, max_num_seqs=max_seqs, max_num_tokens=max_tokens,
          chunked_prefill=chunked, watermark_blocks=watermark)
+
+
+prefix_trace_st = st.lists(st.tuples(st.integers(0, 12), st.integers(0, 2), st.integers(0, 40), st.integers(1, 12)),
+                          min_size=1, max_size=14)
+
+
+@settings(max_examples=200, deadline=None)
+@given(prefix_trace_st, st.integers(4, 40), st.sampled_from([1, 2, 4]), st.integers(1, 6), st.integers(1, 64),
+       st.booleans(), st.integers(0, 2), st.sampled_from([None, 0, 12]))
+def test_cpp_prefix_caching_scheduler_matches_oracle(trace, N, bs, max_seqs, max_tokens, chunked, watermark, ncpu):
+    """Requests with token ids ([CB-PA] §4.2 in the §2.2 loop): prompts share family prefixes, emitted
+    ids are reported each step; plans, cached-token counts, the LRU and the trie agree, with recompute
+    or swap preemption."""
+    prompts = [[fam * 100 + (i % 9) for i in range(12)] + [(r * 13 + i) % 17 for i in range(tail)]
+               for r, (_, fam, tail, _) in enumerate(trace)]
+    t = [(arr, len(prompts[r]), new) for r, (arr, _, _, new) in enumerate(trace)]
+    _run(t, N, bs, 40, cpu_blocks=ncpu, prompts=prompts, max_num_seqs=max_seqs, max_num_tokens=max_tokens,
+         chunked_prefill=chunked, watermark_blocks=watermark)
+
+
+def test_shared_prompt_is_prefilled_once():
+    """Three requests with one 32-token system prompt, arriving one step apart: the second and third
+    find its blocks in the cache and prefill only their own tails; a recomputed request after preemption
+    finds its own blocks again."""
+    system = list(range(100, 132))
+    prompts = [system + [1, 2, 3], system + [4, 5], system + [6] * 9]
+    cs, os_, log = _run([(0, 35, 3), (1, 34, 3), (2, 41, 3)], 64, 8, 20, prompts=prompts, max_num_seqs=4,
+                        max_num_tokens=64)
+    assert os_.cached_tokens == 64 and cs.stats()["cached_tokens"] == 64
+    assert [int(x) for x in log[1]["prefill_ctx"]] == [32] and [int(x) for x in log[2]["prefill_ctx"]] == [32]
 
 
 def test_swap_preemption_keeps_progress():

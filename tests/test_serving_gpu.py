@@ -7,6 +7,8 @@ step writes its rows with reshape_and_cache and runs the prefill and decode
 kernels on the planned tables.  Every output row is checked against the
 float64 oracle's attention over the request's logical K/V (a recomputed
 position gets the same K/V, as recomputation would give)."""
+import zlib
+
 import numpy as np
 import pytest
 import torch
@@ -30,7 +32,35 @@ def test_scheduler_with_swap_preemption_drives_kernels(cuda_ready):
     _serve(swap=True)
 
 
-def _serve(swap):
+def test_scheduler_with_prefix_caching_drives_kernels(cuda_ready):
+    """[CB-PA] §4.2 inside the §2.2 loop: requests share three system prompts and report the ids they
+    generate.  A token's K/V is a function of its whole token prefix (as a model's would be), so a cached
+    block serves every request whose prefix matches; admission skips the cached tokens, and every output
+    row still matches the oracle over each request's own logical K/V."""
+    _serve(swap=False, prefix=True)
+
+
+class _PrefixKV:
+    """Logical K (or V) rows of one request whose row p depends only on its token ids 0..p."""
+
+    def __init__(self, toks, H, D, salt):
+        self.toks, self.H, self.D, self.salt = toks, H, D, salt
+        self.rows = {}
+
+    def row(self, p):
+        key = zlib.crc32(np.asarray(self.toks[:p + 1], np.int32).tobytes())
+        if (p, key) not in self.rows:
+            g = np.random.default_rng([self.salt, p, key])
+            self.rows[(p, key)] = g.standard_normal((self.H, self.D)).astype(np.float16)
+        return self.rows[(p, key)]
+
+    def __getitem__(self, idx):
+        if isinstance(idx, slice):
+            return np.stack([self.row(p) for p in range(*idx.indices(len(self.toks)))])
+        return self.row(idx)
+
+
+def _serve(swap, prefix=False):
     H, D, bs, N = 4, 128, 16, 14            # a pool that forces preemptions
     scale = 1 / np.sqrt(D)
     rng = np.random.default_rng(30)
@@ -38,9 +68,18 @@ def _serve(swap):
     prompts = rng.integers(5, 150, n)
     outs = rng.integers(2, 24, n)
     arrivals = np.sort(rng.integers(0, 6, n))
+    toks = None
+    if prefix:
+        systems = [rng.integers(0, 1000, int(m)).tolist() for m in (40, 57, 64)]
+        toks = [systems[r % 3] + rng.integers(0, 1000, int(rng.integers(1, 40))).tolist() for r in range(n)]
+        prompts = np.asarray([len(t) for t in toks])
     maxlen = int((prompts + outs).max()) + 1
-    K = {r: rng.standard_normal((maxlen, H, D)).astype(np.float16) for r in range(n)}
-    V = {r: rng.standard_normal((maxlen, H, D)).astype(np.float16) for r in range(n)}
+    if prefix:
+        K = {r: _PrefixKV(toks[r], H, D, 1) for r in range(n)}
+        V = {r: _PrefixKV(toks[r], H, D, 2) for r in range(n)}
+    else:
+        K = {r: rng.standard_normal((maxlen, H, D)).astype(np.float16) for r in range(n)}
+        V = {r: rng.standard_normal((maxlen, H, D)).astype(np.float16) for r in range(n)}
     alloc = pk.BlockAllocator(N, bs)
     sched = pk.Scheduler(alloc, max_num_seqs=6, max_num_tokens=64)
     kc = torch.full((N, bs, H, D), float("nan"), dtype=torch.float16, device="cuda")
@@ -58,10 +97,26 @@ def _serve(swap):
     added, checked_rows, preempted, mixed = 0, 0, 0, 0
     for step in range(400):
         while added < n and arrivals[added] <= step:
-            assert sched.add_request(added, int(prompts[added]), int(outs[added])) == pk.PA_OK
+            assert sched.add_request(added, int(prompts[added]), int(outs[added]),
+                                     tokens=None if toks is None else list(toks[added])) == pk.PA_OK
             added += 1
         plan = sched.step()
         preempted += plan["num_preempted"]
+        emitted = []                                        # requests emitting a token this step, in order
+        for r, c, L in zip(plan["prefill_reqs"], plan["prefill_ctx"], plan["prefill_len"]):
+            info = sched.request_info(int(r))[1]
+            if int(c) + int(L) == info["to_prefill"]:
+                emitted.append(int(r))
+        emitted += [int(r) for r in plan["decode_reqs"]]
+
+        def complete():
+            if toks is None:
+                sched.complete()
+                return
+            ids = [int(rng.integers(0, 1000)) for _ in emitted]
+            sched.complete(sampled=ids)
+            for r, t in zip(emitted, ids):
+                toks[r].append(t)
         if swap:
             if len(plan["swap_out"]):
                 pk.swap_blocks(kc, vc, ck, cv, plan["swap_out"], block_bytes, N, NC)
@@ -83,7 +138,7 @@ def _serve(swap):
                     assert np.array_equal(got_v.cpu().numpy().view(np.int16), V[r][:n_kv].view(np.int16)), r
                     swapped_in += 1
         if plan["num_tokens"] == 0:
-            sched.complete()
+            complete()
             if sched.stats()["finished"] == n:
                 break
             continue
@@ -128,7 +183,7 @@ def _serve(swap):
                 ref = oatt.softmax_attention(qd[i][None], K[r][:sl], V[r][:sl], scale)[0]
                 assert np.abs(got[i] - ref).max() <= TOL, (step, r)
                 checked_rows += 1
-        sched.complete()
+        complete()
         if sched.stats()["finished"] == n:
             break
     stats = sched.stats()
@@ -136,6 +191,8 @@ def _serve(swap):
     for r in range(n):
         st, info = sched.request_info(r)
         assert info["generated"] == outs[r]
+    if prefix:
+        assert stats["cached_tokens"] > 0 and alloc.cache_stats()["hit_blocks"] > 0
     if swap:
         assert stats["swap_outs"] > 0 and stats["swap_ins"] == stats["swap_outs"] and swapped_in > 0
         assert stats["prefill_tokens"] == int(prompts.sum())      # nothing was recomputed
