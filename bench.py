@@ -549,9 +549,20 @@ def serve_trace(n, seed=2060):
     return prompts, outs
 
 
+def shared_prompt_tokens(prompts, n_systems, system_len, seed=4383):
+    """Token ids for the trace's prompts: request r starts with one of n_systems shared system prompts of
+    system_len tokens (round robin) and continues with its own ids; its prompt length grows by system_len."""
+    rng = np.random.default_rng(seed)
+    systems = [rng.integers(0, 32000, system_len).astype(np.int32) for _ in range(n_systems)]
+    return [np.concatenate([systems[r % n_systems], rng.integers(0, 32000, int(p)).astype(np.int32)])
+            for r, p in enumerate(prompts)]
+
+
 def run_serve(args):
     """Continuous batching over a seeded trace: the C++ scheduler plans every step, the step runs
-    reshape_and_cache, the chunked-prefill kernel and the decode kernel for one attention layer."""
+    reshape_and_cache, the chunked-prefill kernel and the decode kernel for one attention layer.  With
+    --serve-system-prompt L, every prompt starts with one of 8 shared L-token system prompts and goes
+    through the prefix cache (its token ids are given; emitted ids are reported each step)."""
     import torch
 
     import paged_kv_cache_411_b200 as pk
@@ -561,12 +572,17 @@ def run_serve(args):
     H, D, bs = 32, 128, 16
     n = args.serve_requests
     prompts, outs = serve_trace(n)
+    toks = None
+    if args.serve_system_prompt:
+        toks = shared_prompt_tokens(prompts, 8, args.serve_system_prompt)
+        prompts = prompts + args.serve_system_prompt
     max_seqs, max_tokens = 256, 8192
     N = args.serve_blocks
     alloc = pk.BlockAllocator(N, bs)
     sched = pk.Scheduler(alloc, max_num_seqs=max_seqs, max_num_tokens=max_tokens)
     for r in range(n):
-        sched.add_request(r, int(prompts[r]), int(outs[r]))
+        sched.add_request(r, int(prompts[r]), int(outs[r]), tokens=None if toks is None else toks[r])
+    id_rng = np.random.default_rng(198203)
     kc = torch.zeros((N, bs, H, D), dtype=torch.float16, device=dev)
     vc = torch.zeros_like(kc)
     g = torch.Generator(device=dev).manual_seed(7)
@@ -635,7 +651,13 @@ def run_serve(args):
             ev1.record(stream)
             stream.synchronize()                     # the step's result goes back to the host
             gpu_ms.append(ev0.elapsed_time(ev1))
-        sched.complete()
+        if toks is None:
+            sched.complete()
+        else:
+            # one id per emitted token (requests whose prefill completed, then the decodes)
+            n_emit = S + int(sum(1 for r, c, L in zip(plan["prefill_reqs"], plan["prefill_ctx"], plan["prefill_len"])
+                                 if c + L == sched.request_info(int(r))[1]["to_prefill"]))
+            sched.complete(sampled=id_rng.integers(0, 32000, n_emit))
         ends.append(time.perf_counter() - t_start)
     wall = time.perf_counter() - t_start
     ends = np.asarray(ends)
@@ -656,7 +678,9 @@ def run_serve(args):
         "metric": "serve: output tokens/s of continuous batching over one attention layer", "impl": "ours",
         "value": round(float(outs.sum()) / wall, 1), "unit": "tok/s", "higher_is_better": True,
         "data": "synthetic", "dtype": "f16",
-        "config": {"workload": f"serve_trace_{n}req_rate_inf_lognormal223_198", "num_heads": H, "head_dim": D,
+        "config": {"workload": f"serve_trace_{n}req_rate_inf_lognormal223_198"
+                   + (f"_system_prompt{args.serve_system_prompt}x8" if toks is not None else ""),
+                   "num_heads": H, "head_dim": D,
                    "block_size": bs, "num_blocks": N, "max_num_seqs": max_seqs, "max_num_batched_tokens": max_tokens,
                    "chunked_prefill": True, "input_tokens": int(prompts.sum()), "output_tokens": int(outs.sum())},
         "wall_s": round(wall, 3), "req_per_s": round(n / wall, 2), "steps": st["steps"],
@@ -664,6 +688,12 @@ def run_serve(args):
         "gpu_ms_total": round(float(np.sum(gpu_ms)), 2), "host_schedule_s": round(host_s, 3),
         "ttft_ms": dist(ttft), "tpot_ms": dist(tpot),
     }
+    if toks is not None:
+        cs = alloc.cache_stats()
+        line["prefix_cache"] = {"cached_prompt_tokens": st["cached_tokens"], "prompt_tokens": int(prompts.sum()),
+                                "hit_rate": round(st["cached_tokens"] / float(prompts.sum()), 4),
+                                "hit_blocks": cs["hit_blocks"], "evictions": cs["evictions"],
+                                "prefix_nodes_at_end": cs["prefix_nodes"], "cached_blocks_at_end": cs["cached_blocks"]}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -684,6 +714,8 @@ def main(argv=None):
                     help="continuous-batching run over a seeded trace instead of the single-step benchmark")
     ap.add_argument("--serve-requests", type=int, default=1000)
     ap.add_argument("--serve-blocks", type=int, default=7680)
+    ap.add_argument("--serve-system-prompt", type=int, default=0,
+                    help="serve: prefix every prompt with one of 8 shared system prompts of this many tokens")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")

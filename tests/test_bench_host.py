@@ -34,6 +34,27 @@ def test_prefill_flops_mixed():
     assert bench.prefill_flops(w) == 917_760 * 4 * 32 * 128 == 15_036_579_840
 
 
+def test_shared_prefix_counted_once_in_unique_bytes():
+    # 8 sequences share a 1024-token prefix (32 whole blocks of 32): 7 of the 8 reads of it are not unique
+    w = si.get("longctx")
+    extra = bench.shared_prefix_rereads(w, w.decode_lens)
+    assert extra == 7 * 1024 * 32 * 128 * 2 * 2
+    dec, _, _ = bench.step_bytes(w, w.decode_lens, 1024, 8)
+    assert dec - extra == dec - 7 * 16 * 2**20     # 16 MiB of K+V per 1024 tokens x 32 heads x 128
+    assert bench.shared_prefix_rereads(si.get("b256"), si.get("b256").decode_lens) == 0
+
+
+def test_prefill_8k_flops():
+    w = si.get("prefill8k")
+    assert bench.prefill_flops(w) == 4 * 32 * 128 * (8192 * 8193 // 2)
+
+
+def test_timing_distribution():
+    d = bench.dist_ms([1.0, 2.0, 3.0, 4.0, 100.0])
+    assert d["median"] == 3.0 and d["n"] == 5 and d["mean"] == 22.0
+    assert d["p10"] == pytest.approx(1.4) and d["p90"] == pytest.approx(61.6)
+
+
 def test_oracle_sample_is_bounded_and_seeded():
     w = si.get("b256")
     a = bench.oracle_sample_seqs(w, 12000)
