@@ -44,6 +44,7 @@
 // fixed, so the result does not depend on physical block placement (bitwise)
 // nor on which CTA ran which item.
 #include <algorithm>
+#include <type_traits>
 #include <mutex>
 
 #include "device_common.cuh"
@@ -196,7 +197,7 @@ __device__ __forceinline__ float reduce_scores(float (&v)[NV], int lane) {
 }
 
 // ------------------------------------------------------------------ plan ----
-__global__ void __launch_bounds__(1024) decode_plan_kernel(DecodeParams p, int32_t hg_count,
+__global__ void __launch_bounds__(256) decode_plan_kernel(DecodeParams p, int32_t hg_count,
                                                            int32_t target_items, int32_t max_split,
                                                            int32_t head_dim) {
     constexpr int kNC = 4;
@@ -302,6 +303,8 @@ template <int D>
 __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
     pdl_wait();
     constexpr int VEC = D / 32;
+    constexpr int kBatch = 8;                   // partitions whose loads are in flight together
+    using Vec = typename std::conditional<VEC == 4, float4, float2>::type;
     const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (gw >= p.S * p.H) return;
@@ -315,15 +318,25 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
     float L = 0.f, acc[VEC];
 #pragma unroll
     for (int k = 0; k < VEC; ++k) acc[k] = 0.f;
-#pragma unroll 4
-    for (int i = 0; i < n; ++i) {
-        const int64_t pi = base + static_cast<int64_t>(i) * p.H;
-        const float2 ml = p.part_ml[pi];
-        const float w = exp2f(ml.x - M);
-        L = fmaf(ml.y, w, L);
-        const float* a = p.part_acc + pi * D + lane * VEC;
+    for (int i0 = 0; i0 < n; i0 += kBatch) {
+        // every load of the batch first, then the merge in partition order
+        float2 ml[kBatch];
+        Vec a[kBatch];
 #pragma unroll
-        for (int k = 0; k < VEC; ++k) acc[k] = fmaf(a[k], w, acc[k]);
+        for (int b = 0; b < kBatch; ++b) {
+            const int64_t pi = base + static_cast<int64_t>(min(i0 + b, n - 1)) * p.H;
+            ml[b] = p.part_ml[pi];
+            a[b] = *reinterpret_cast<const Vec*>(p.part_acc + pi * D + lane * VEC);
+        }
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            if (i0 + b >= n) break;
+            const float w = exp2f(ml[b].x - M);
+            L = fmaf(ml[b].y, w, L);
+            const float* av = reinterpret_cast<const float*>(&a[b]);
+#pragma unroll
+            for (int k = 0; k < VEC; ++k) acc[k] = fmaf(av[k], w, acc[k]);
+        }
     }
     const float r = 1.f / L;
     __half* o = p.out + static_cast<int64_t>(gw) * D + lane * VEC;
@@ -730,7 +743,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream, const char**
     {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(1);
-        cfg.blockDim = dim3(1024);
+        cfg.blockDim = dim3(256);
         cfg.stream = stream;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
