@@ -8,39 +8,48 @@
 // decode steps; §1.1: prefill is the compute-bound phase) over the paged read
 // of §3.3.  The chunk's own K/V must already be in the pool.
 //
-// One CTA computes one tile of 128 query rows x one head (FlashAttention
-// order, online softmax over 128-key tiles):
-//   * kIssueWarps K warps and kIssueWarps V warps (producers, from warp 8) load
-//     the Q tile once and stream the K and the V tiles into two-stage rings
-//     with TMA: a tile of 128 keys is gathered from the paged pool with one 3-D
-//     box per (physical block, 64-dim chunk) ([box rows][1 head][64 dims],
-//     128-byte swizzle), landing directly in the canonical UMMA layout; the
-//     boxes are dealt to the lanes of the operand's warps, one each, and the
-//     next tile's block ids are read a tile ahead;
-//   * the last warp (one elected thread) issues tcgen05.mma: S = Q K^T (A and B
-//     K-major) into a double-buffered fp32 TMEM tile, and P V (A = P read from
-//     TMEM, B MN-major straight from the V tile) accumulated in TMEM across all
-//     key tiles as two partial outputs, O_0 over the first 64 keys of every
-//     tile and O_1 over the last 64; completions are signalled with
-//     tcgen05.commit on mbarriers;
-//   * warps 0-7 (two threads per query row = per TMEM lane; thread g of a row
-//     owns key columns g*64 .. g*64+63 of every tile and so the partial output
-//     O_g) read S with tcgen05.ld, apply the causal mask on the diagonal tiles
-//     and run the online softmax of their half on their own: each keeps its own
-//     running max m_g and sum l_g, and P = 2^(s*scale*log2e - m_g) is written
-//     as fp16 pairs over the first half of the thread's own S columns in TMEM,
-//     where the P V MMA reads it (shared memory carries only Q, K and V).
-//     m_g only moves when a tile's max exceeds it by more than kRescaleLog2
-//     (P then stays <= 2^kRescaleLog2, exact in fp16 up to its 11-bit
-//     mantissa); when it moves, the warp rescales its rows of O_g in TMEM
-//     (after the previous P V has completed) before the next P V adds to it.
-//     The two halves of a row are merged once, after the last tile:
-//     O = (O_0 2^(m_0-M) + O_1 2^(m_1-M)) / (l_0 2^(m_0-M) + l_1 2^(m_1-M)),
-//     M = max(m_0, m_1).  The MMA of tile j+1 overlaps the softmax of tile j.
-// Keys past the tile's last query position are masked; rows of V past the
-// sequence end are zeroed before P.V so stale or poisoned pool rows never
-// reach the MMA.  Every wait is bounded; on a timeout the CTA records
-// PA_DEVCHK_TIMEOUT, lets its copies and MMAs drain, frees its TMEM and exits.
+// One CTA computes 256 query rows of one head as two 128-row query tiles, Q0
+// and Q1, that share every K and V tile (FlashAttention order, online softmax
+// over 128-key tiles).  The two tiles exist so that the tensor core always has
+// independent work queued: while softmax warpgroup 0 turns S0(j) into P0(j),
+// the tensor core runs P1(j-1) V and S1(j), and the other way round.
+//   * Producers (warp 8: K, warp 9: V; warp 8 also loads Q0 and Q1 once)
+//     stream 128-key tiles into two-stage rings with TMA.  A tile is gathered
+//     from the paged pool with one 3-D box per (physical block, 64-dim chunk)
+//     ([box rows][1 head][64 dims], 128-byte swizzle), landing directly in the
+//     canonical UMMA layouts; each lane issues one box and reads the block id
+//     of its box of the next tile a tile ahead.  After the last V tile has
+//     landed, the V warp zeroes its rows past the sequence end (pool rows
+//     there may hold anything, and 0 * NaN would poison P V).
+//   * MMA issuer (warp 10, one thread): tcgen05.mma kind::f16 with fp32
+//     accumulators in TMEM.  S_g(j) = Q_g K_j^T into the tile's S buffer;
+//     O_g += P_g(j) V_j with A = P_g read from TMEM (fp16, over the first half
+//     of the S buffer) and B = V_j from shared memory.  Issue order per key
+//     tile: P0 V, S0(j+1), P1 V, S1(j+1); a commit after each group signals the
+//     softmax warps (S landed, P V landed) and the producers (K / V stage free).
+//   * Softmax warpgroups 0 and 1 (warps 0-3 and 4-7; one thread per query row
+//     = TMEM lane): read the 128 scores of S_g(j) with tcgen05.ld into
+//     registers (11 warps leave each thread 168), take the row max (causal
+//     mask on the diagonal tiles only), and write P = 2^(s*scale*log2e - m) as
+//     fp16 pairs over the first half of the S buffer with tcgen05.st.  The running
+//     max m only moves when a tile's max exceeds it by more than kRescaleLog2
+//     (P then stays <= 2^kRescaleLog2, exact in fp16 to its 11-bit mantissa);
+//     when it moves, the warp rescales its rows of O_g in TMEM after the
+//     previous P V has landed and before the next one is issued.  The scaling
+//     runs in packed f32x2 arithmetic, the row max takes three operands per
+//     instruction, and the row sum adds the same fp16 values of P that the P V
+//     MMA adds.  After the last tile each thread normalises its row of O_g and
+//     stores it as fp16.
+// When a launch has too few (256-row query block, head) pairs to fill the GPU
+// (a short chunk after a long cached prefix), it runs in clusters of two CTAs
+// per pair instead: each CTA takes half of the key tiles, and the two partial
+// results of every row, (O, m, l), are merged with the log-sum-exp rule
+// through distributed shared memory at the end (no workspace, no second
+// launch); CTA c of the cluster finalises query tile c.
+// Every wait is bounded; on a timeout the CTA records PA_DEVCHK_TIMEOUT, lets
+// its copies and MMAs drain, frees its TMEM and exits.
+#include <algorithm>
+#include <cstdlib>
 #include <mutex>
 
 #include "device_common.cuh"
@@ -49,15 +58,17 @@
 namespace pagedkv {
 namespace {
 
-constexpr int kTile = 128;
-constexpr int kSoftmaxWarps = 8;          // two warpgroups: each owns half of the key columns of S
-constexpr int kIssueWarps = 2;                        // TMA-issuing warps per operand (K, V)
-constexpr int kFirstKWarp = 8;                        // K warps (the first also loads Q)
+constexpr int kTile = 128;                      // query rows of a query tile = keys of a key tile
+constexpr int kQTiles = 2;                      // query tiles per CTA, one softmax warpgroup each
+constexpr int kRowsPerCta = kQTiles * kTile;
+constexpr int kSoftmaxWarps = 4 * kQTiles;
+constexpr int kIssueWarps = 1;                  // TMA-issuing warps per operand (K, V)
+constexpr int kFirstKWarp = kSoftmaxWarps;      // K warps (the first also loads Q)
 constexpr int kFirstVWarp = kFirstKWarp + kIssueWarps;
 constexpr int kMmaWarp = kFirstVWarp + kIssueWarps;
 constexpr int kThreadsP = (kMmaWarp + 1) * 32;
 constexpr float kLog2eP = 1.4426950408889634f;
-// A thread's running max (log2 domain) is raised only when a tile's max exceeds it by more than this;
+// A row's running max (log2 domain) is raised only when a tile's max exceeds it by more than this;
 // P <= 2^kRescaleLog2 = 256 is exact enough in fp16 and far from its overflow.
 constexpr float kRescaleLog2 = 8.f;
 
@@ -66,7 +77,7 @@ struct PrefillParams {
     const int32_t* block_tables;
     const int32_t* q_start;
     const int32_t* ctx_before;
-    int32_t B, T, H, max_blocks, bs, num_blocks, grid_tiles, box_rows;
+    int32_t B, T, H, max_blocks, bs, num_blocks, grid_blocks, box_rows;
     float qscale;
     int32_t* err_flag;
     uint64_t wait_ns;          // limit of every pipeline wait (kWaitLimitNs by default)
@@ -79,29 +90,57 @@ struct PCfg {
     static constexpr int kChunkBytes = kTile * 128;               // 128 rows x 128 B = 16 KB
     static constexpr int kOpBytes = kChunks * kChunkBytes;        // one Q, K or V tile
     static constexpr int kStages = 2;
-    static constexpr size_t kOffQ = 0;
-    static constexpr size_t kOffK = kOffQ + kOpBytes;
+    static constexpr size_t kOffQ = 0;                            // Q0, Q1
+    static constexpr size_t kOffK = kOffQ + size_t(kQTiles) * kOpBytes;
     static constexpr size_t kOffV = kOffK + size_t(kStages) * kOpBytes;
     static constexpr size_t kOffBar = kOffV + size_t(kStages) * kOpBytes;
-    static constexpr int kNumBars = 13;
+    static constexpr int kNumBars = 18;
     static constexpr size_t kOffSlot = kOffBar + kNumBars * 8;
-    static constexpr size_t kOffRed = kOffSlot + 64;                 // final exchange: maxes [2][128], sums [2][128]
     // Every CTA takes all 512 TMEM columns, so the request is kept above half the SM's shared
     // memory: one CTA per SM, and tcgen05.alloc never has to wait for a neighbour.
-    static constexpr size_t kSmemUsed = kOffRed + 4 * 128 * 4 + 1024;
+    static constexpr size_t kSmemUsed = kOffSlot + 64 + 1024;
     static constexpr size_t kSmemBytes = kSmemUsed > 120 * 1024 ? kSmemUsed : 120 * 1024;
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kColS = 0;                          // S buffers: columns 0 and 128
-    static constexpr uint32_t kColO = 256;                        // O_0 at 256, O_1 at 256 + D
+    static constexpr uint32_t kColS = 0;                          // S_g at g * 128 (P_g over its first 64)
+    static constexpr uint32_t kColO = kQTiles * kTile;            // O_g at 256 + g * D
+    static_assert(kColO + kQTiles * D <= kTmemCols, "TMEM budget");
+    static_assert(kSmemUsed <= 227 * 1024, "shared-memory budget");
 };
 
-__device__ __forceinline__ void st_shared_u4(void* p, uint4 v) {
-    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(p)), "r"(v.x), "r"(v.y), "r"(v.z),
-                 "r"(v.w)
-                 : "memory");
+__device__ __forceinline__ void st_shared_zero16(uint32_t addr) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0) : "memory");
 }
 
-template <int D>
+// ---- thread-block cluster (split key range): the two CTAs of a cluster exchange partial rows
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Every thread of both CTAs arrives (release) and waits (acquire): shared-memory writes made before it,
+// local or remote, are visible after it.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// The shared::cluster address of this CTA's shared-memory address `a` in the cluster's CTA `rank`.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t a, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_cluster_f4(uint32_t addr, float a, float b, float c, float d) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+__device__ __forceinline__ void st_cluster_f2(uint32_t addr, float a, float b) {
+    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
+}
+
+// SPLIT == 2: the kernel is launched in clusters of two CTAs that share one (query block, head); CTA c of
+// the cluster runs key tiles [jb, je) (the first or the second half of the key range), and the two partial
+// results of every row are merged through distributed shared memory at the end, CTA c finalising query
+// tile c.  Used when the launch has too few (query block, head) pairs to fill the GPU.
+template <int D, int SPLIT>
 __global__ void __launch_bounds__(kThreadsP, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, PrefillParams p) {
@@ -113,23 +152,28 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint8_t* sV = smem + C::kOffV;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* q_full = bars + 0;
-    uint64_t* k_full = bars + 1;     // [2]
-    uint64_t* v_full = bars + 3;     // [2]
-    uint64_t* s_full = bars + 5;     // [2] S(j) is in TMEM, which also frees K stage j % 2
-    uint64_t* p_full = bars + 7;
-    uint64_t* pv_done = bars + 8;    // [2] P.V(j) has landed in O_0/O_1, which also frees V stage j % 2
-    uint64_t* drain = bars + 10;
-    uint64_t* sum_bar = bars + 11;   // final (max, sum) exchange between the two halves of a row
-    uint64_t* never = bars + 12;     // no thread ever arrives on it (failure-detection test)
+    uint64_t* k_full = bars + 1;     // [2] K stage landed
+    uint64_t* k_empty = bars + 3;    // [2] every S MMA reading the K stage has completed
+    uint64_t* v_full = bars + 5;     // [2] V stage landed
+    uint64_t* v_empty = bars + 7;    // [2] every P V MMA reading the V stage has completed
+    uint64_t* v_tail = bars + 9;     // the last V tile's rows past the sequence end are zero
+    uint64_t* s_full = bars + 10;    // [g] S_g(j) is in TMEM
+    uint64_t* p_full = bars + 12;    // [g] P_g(j) is in TMEM (and O_g rescaled if needed)
+    uint64_t* pv_done = bars + 14;   // [g] O_g += P_g(j) V_j has landed
+    uint64_t* drain = bars + 16;
+    uint64_t* never = bars + 17;     // no thread ever arrives on it (failure-detection test)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffSlot);
-    volatile int* info = reinterpret_cast<volatile int*>(smem + C::kOffSlot + 16);   // b, qt, abort
+    volatile int* info = reinterpret_cast<volatile int*>(smem + C::kOffSlot + 16);   // b, qb, abort
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = blockIdx.y;
+    const unsigned work = blockIdx.x / SPLIT;           // the two CTAs of a cluster share their work item
+    const int crank = SPLIT == 2 ? static_cast<int>(cluster_ctarank()) : 0;
+    const int h = static_cast<int>(work % static_cast<unsigned>(p.H));
+    const int rank = static_cast<int>(work / static_cast<unsigned>(p.H));
 
     if (threadIdx.x == 0) {
-        int g = p.grid_tiles - 1 - static_cast<int>(blockIdx.x);   // heaviest (latest) tiles first
-        int bsel = -1, qt = 0;
+        int g = p.grid_blocks - 1 - rank;        // the latest (heaviest) query blocks go first
+        int bsel = -1, qb = 0;
         for (int b = 0; b < p.B; ++b) {
             const int s0 = p.q_start[b], s1 = p.q_start[b + 1];
             if (s0 < 0 || s1 < s0 || s1 > p.T) {
@@ -137,9 +181,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 bsel = -1;
                 break;
             }
-            const int nt = (s1 - s0 + kTile - 1) / kTile;
-            if (bsel < 0 && g >= 0 && g < nt) { bsel = b; qt = g; }
-            g -= nt;
+            const int nb = (s1 - s0 + kRowsPerCta - 1) / kRowsPerCta;
+            if (bsel < 0 && g >= 0 && g < nb) { bsel = b; qb = g; }
+            g -= nb;
         }
         if (bsel >= 0) {
             const int L = p.q_start[bsel + 1] - p.q_start[bsel];
@@ -150,32 +194,50 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
         }
         info[0] = bsel;
-        info[1] = qt;
+        info[1] = qb;
         info[2] = 0;
         mbar_init(q_full, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&k_full[i], kIssueWarps);
             mbar_init(&v_full[i], kIssueWarps);
+            mbar_init(&k_empty[i], 1);
+            mbar_init(&v_empty[i], 1);
             mbar_init(&s_full[i], 1);
+            mbar_init(&p_full[i], 4);
             mbar_init(&pv_done[i], 1);
         }
-        mbar_init(p_full, kSoftmaxWarps);
+        mbar_init(v_tail, 1);
         mbar_init(drain, 1);
-        mbar_init(sum_bar, kSoftmaxWarps);
         mbar_init(never, 1);
         mbar_init_fence();
     }
     __syncthreads();
     const int b = info[0];
-    if (b < 0) return;                                  // uniform: no tile for this CTA
-    const int qt = info[1];
+    if (b < 0) return;                                  // uniform: no work for this CTA
+    const int qb = info[1];
     const int s0 = p.q_start[b];
     const int L = p.q_start[b + 1] - s0;
     const int ctx = p.ctx_before[b];
-    const int q0 = s0 + qt * kTile;                     // first query row of the tile
-    const int rows = min(kTile, L - qt * kTile);
-    const int kv_len = ctx + qt * kTile + rows;         // keys 0 .. kv_len-1 are visible to some row
-    const int n_tiles = (kv_len + kTile - 1) / kTile;
+    const int row0 = qb * kRowsPerCta;                  // first row of Q0 within the request
+    const int q0 = s0 + row0;                           // ... within q / out
+    // query tile g: its valid rows, the keys its last valid row sees, and the key tiles that covers
+    int rows_g[kQTiles], kvl_g[kQTiles], n_g[kQTiles];
+#pragma unroll
+    for (int g = 0; g < kQTiles; ++g) {
+        rows_g[g] = max(0, min(kTile, L - row0 - g * kTile));
+        kvl_g[g] = rows_g[g] > 0 ? ctx + row0 + g * kTile + rows_g[g] : 0;
+        n_g[g] = (kvl_g[g] + kTile - 1) / kTile;
+    }
+    const int kv_len = max(kvl_g[0], kvl_g[1]);
+    const int n_tiles = max(n_g[0], n_g[1]);            // >= 1: Q0 always has a valid row
+    // this CTA's key tiles [jb, je): all of them, or one half of them in a split cluster
+    const int half = (n_tiles + 1) / 2;
+    const int jb = (SPLIT == 2 && crank == 1) ? half : 0;
+    const int je = (SPLIT == 2 && crank == 0) ? half : n_tiles;
+    const int n_loc = je - jb;                          // may be 0 (the second CTA of a one-tile block)
+    int je_g[kQTiles];                                  // query tile g's key tiles here: [jb, je_g)
+#pragma unroll
+    for (int g = 0; g < kQTiles; ++g) je_g[g] = max(jb, min(je, n_g[g]));
 
     if (warp == kMmaWarp) {
         tmem_alloc(tmem_slot, C::kTmemCols);
@@ -190,6 +252,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         flag_error(p.err_flag, kDevchkTimeout);
         info[2] = 1;
     };
+    // a softmax thread's partial result for the split merge: running max, sum, its tile count, no timeout
+    float sm_m = -INFINITY, sm_l = 0.f;
+    int sm_cnt = 0;
+    bool sm_ok = false;
 
     if (warp >= kFirstKWarp && warp < kMmaWarp) {
         // ======================================================= TMA producers (K warps, V warps)
@@ -202,17 +268,20 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int wsub = warp - (is_k ? kFirstKWarp : kFirstVWarp);
         const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
         uint64_t* full = is_k ? k_full : v_full;
-        uint64_t* empty = is_k ? s_full : pv_done;      // stage j % 2 is free once S / P.V of tile j-2 is done
+        uint64_t* empty = is_k ? k_empty : v_empty;
         uint8_t* base = is_k ? sK : sV;
-        const uint64_t pol = l2_policy_evict_last();     // K/V tiles are re-read by the head's other q-tiles
+        const uint64_t pol = l2_policy_evict_last();     // K/V tiles are re-read by the head's other CTAs
         if (lane == 0) {
             tma_prefetch_desc(tm);
-            if (is_k && wsub == 0) {
+            if (is_k && wsub == 0 && n_loc > 0) {
                 tma_prefetch_desc(&tm_q);
-                mbar_arrive_expect_tx(q_full, C::kOpBytes);
+                mbar_arrive_expect_tx(q_full, kQTiles * C::kOpBytes);
 #pragma unroll
-                for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_3d(sQ + c * C::kChunkBytes, &tm_q, q_full, c * 64, h, q0, pol);
+                for (int g = 0; g < kQTiles; ++g)
+#pragma unroll
+                    for (int c = 0; c < C::kChunks; ++c)
+                        tma_load_3d(sQ + g * C::kOpBytes + c * C::kChunkBytes, &tm_q, q_full, c * 64, h,
+                                    q0 + g * kTile, pol);
             }
         }
         const int br = p.box_rows;
@@ -221,17 +290,18 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int box = my_i / C::kChunks, chunk = my_i % C::kChunks;
         auto nbox_of = [&](int j) { return (min(kTile, kv_len - j * kTile) + br - 1) / br; };
         auto read_id = [&](int j) -> int {               // raw table entry; checked at use
-            return (j < n_tiles && box < nbox_of(j)) ? p.block_tables[tbase + (j * kTile + box * br) / p.bs] : 0;
+            return (j < je && box < nbox_of(j)) ? p.block_tables[tbase + (j * kTile + box * br) / p.bs] : 0;
         };
-        int last = -1;                                   // last tile whose copies this warp issued
-        int bid = read_id(0);
-        for (int j = 0; j < n_tiles; ++j) {
-            const int st = j & 1;
+        int last = -1;                                   // last ring slot (local tile index) this warp filled
+        int bid = read_id(jb);
+        for (int j = jb; j < je; ++j) {
+            const int i = j - jb;                        // ring position
+            const int st = i & 1;
             const int nbox = nbox_of(j);
             const int bid_next = read_id(j + 1);
             const int n_mine = (nbox * C::kChunks - wsub + kIssueWarps - 1) / kIssueWarps;
             const uint32_t bytes = static_cast<uint32_t>(n_mine * br * 128);
-            if (!mbar_wait(&empty[st], ((j >> 1) & 1) ^ 1, p.wait_ns)) { abort_now(); break; }
+            if (!mbar_wait(&empty[st], ((i >> 1) & 1) ^ 1, p.wait_ns)) { abort_now(); break; }
             if (info[2]) break;
             if (lane == 0) mbar_arrive_expect_tx(&full[st], bytes);
             __syncwarp();
@@ -245,8 +315,27 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 tma_load_3d(base + st * C::kOpBytes + chunk * C::kChunkBytes + box * br * 128, tm, &full[st],
                             chunk * 64, h, my_bid * p.bs + key % p.bs, pol);
             }
-            last = j;
+            last = i;
             bid = bid_next;
+        }
+        if (!is_k && wsub == 0 && !info[2] && je == n_tiles && n_loc > 0) {
+            // the last V tile: rows past the sequence end become zero before any P V reads them
+            const int jl = n_tiles - 1, il = jl - jb;
+            if (mbar_wait(&v_full[il & 1], (il >> 1) & 1, p.wait_ns)) {
+                const int valid = kv_len - jl * kTile;                 // 1 .. 128
+                const int units = (kTile - valid) * C::kChunks * 8;   // 16-byte units to clear
+                const uint32_t vbase = smem_u32(sV + (il & 1) * C::kOpBytes);
+                for (int u = lane; u < units; u += 32) {
+                    const int row = valid + u / (C::kChunks * 8);
+                    const int rem = u % (C::kChunks * 8);
+                    st_shared_zero16(vbase + (rem >> 3) * C::kChunkBytes + row * 128 + (rem & 7) * 16);
+                }
+                fence_proxy_async_smem();                  // the zeros reach the tensor core's view
+                __syncwarp();
+                if (lane == 0) mbar_arrive(v_tail);
+            } else {
+                abort_now();
+            }
         }
         if (info[2]) {
             // unwind: let the copies this warp issued land
@@ -261,177 +350,185 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const uint64_t dQ = umma_desc_sw128(smem_u32(sQ), 16, 1024);
             const uint64_t dK = umma_desc_sw128(smem_u32(sK), 16, 1024);
             const uint64_t dV = umma_desc_sw128(smem_u32(sV), C::kChunkBytes, 1024);
-            bool ok = mbar_wait(q_full, 0, p.wait_ns);
+            const int n0 = n_g[0], n1 = n_g[1];
             // An mbarrier answers after ~150 cycles even when its phase is complete, so this thread asks
             // early (mbar_test_wait) and collects the answers after the MMAs it issues meanwhile; it only
             // blocks when a phase really is still open.
-            auto issue_s = [&](int j, bool k_ready) -> bool {
-                const int st = j & 1;
-                if (!k_ready && !mbar_wait(&k_full[st], (j >> 1) & 1, p.wait_ns)) return false;
-                // S(j) reuses the buffer of S(j-2)/P(j-2): it is issued after P.V(j-2), which the
-                // tensor core runs first, and P.V(j-2) waited for every softmax warp to finish that tile
-                tc_fence_after_sync();
-                const uint32_t d = tmem + C::kColS + (j & 1) * kTile;
-                const uint64_t dKs = umma_desc_advance(dK, st * C::kOpBytes);
+            // i: the tile's ring position (its index among this CTA's key tiles)
+            auto issue_s = [&](int g, int i) {
+                const uint32_t d = tmem + C::kColS + g * kTile;
+                const uint64_t dQg = umma_desc_advance(dQ, g * C::kOpBytes);
+                const uint64_t dKs = umma_desc_advance(dK, (i & 1) * C::kOpBytes);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-                    umma_f16_ss(d, umma_desc_advance(dQ, off), umma_desc_advance(dKs, off), idesc_qk, kk > 0);
+                    umma_f16_ss(d, umma_desc_advance(dQg, off), umma_desc_advance(dKs, off), idesc_qk, kk > 0);
                 }
-                umma_commit(&s_full[st]);
-                return true;
+                umma_commit(&s_full[g]);
             };
-            if (ok) ok = issue_s(0, false);
-            bool k_ready = ok && n_tiles > 1 && mbar_test_wait(&k_full[1], 0);
-            for (int j = 0; ok && j < n_tiles; ++j) {
-                const int st = j & 1;
-                const bool p_ready = mbar_test_wait(p_full, j & 1);
-                const bool v_ready = mbar_test_wait(&v_full[st], (j >> 1) & 1);
-                if (j + 1 < n_tiles && !(ok = issue_s(j + 1, k_ready))) break;
-                if (!p_ready && !(ok = mbar_wait(p_full, j & 1, p.wait_ns))) break;
-                if (!v_ready && !(ok = mbar_wait(&v_full[st], (j >> 1) & 1, p.wait_ns))) break;
-                if (info[2]) { ok = false; break; }
-                k_ready = j + 2 < n_tiles && mbar_test_wait(&k_full[st], ((j + 2) >> 1) & 1);   // for S(j+2)
-                tc_fence_after_sync();
-                const uint64_t dVs = umma_desc_advance(dV, st * C::kOpBytes);
-                const uint32_t pbase = tmem + C::kColS + (j & 1) * kTile;
+            auto issue_pv = [&](int g, int i) {
+                // P_g of keys 16kk .. 16kk+15 is fp16 in columns 8kk .. 8kk+7 of the tile's S buffer
+                const uint32_t o = tmem + C::kColO + g * D;
+                const uint32_t pbase = tmem + C::kColS + g * kTile;
+                const uint64_t dVs = umma_desc_advance(dV, (i & 1) * C::kOpBytes);
 #pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk) {
-                    // keys 0-63 of the tile add to O_0, keys 64-127 to O_1; tile 0 starts both.  P of
-                    // keys 64h .. 64h+63 is fp16 in columns 64h .. 64h+31 of the tile's S buffer.
-                    const uint32_t d = tmem + C::kColO + (kk >> 2) * D;
-                    const uint32_t pa = pbase + (kk >> 2) * 64 + (kk & 3) * 8;
-                    umma_f16_ts(d, pa, umma_desc_advance(dVs, kk * 16 * 128), idesc_pv, j > 0 || (kk & 3) != 0);
+                for (int kk = 0; kk < kTile / 16; ++kk)
+                    umma_f16_ts(o, pbase + kk * 8, umma_desc_advance(dVs, kk * 16 * 128), idesc_pv, i > 0 || kk > 0);
+                umma_commit(&pv_done[g]);
+            };
+            bool ok = n_loc == 0 || (mbar_wait(q_full, 0, p.wait_ns) && mbar_wait(&k_full[0], 0, p.wait_ns));
+            if (ok && n_loc > 0) {
+                tc_fence_after_sync();
+                if (jb < n0) issue_s(0, 0);
+                if (jb < n1) issue_s(1, 0);
+                umma_commit(&k_empty[0]);
+            }
+            for (int i = 0; ok && i < n_loc; ++i) {
+                const int j = jb + i;                       // the key tile
+                const int st = i & 1;
+                const bool next = i + 1 < n_loc;
+                // each ring barrier is waited on once per tile, right before the first MMA that needs it
+                bool k_ready = !next, v_ready = false, tail_ready = j != n_tiles - 1;
+                if (info[2]) { ok = false; break; }
+#pragma unroll
+                for (int g = 0; g < kQTiles; ++g) {
+                    if (j >= je_g[g]) continue;
+                    if (!(ok = mbar_wait(&p_full[g], i & 1, p.wait_ns))) break;
+                    if (!v_ready && !(ok = mbar_wait(&v_full[st], (i >> 1) & 1, p.wait_ns))) break;
+                    v_ready = true;
+                    if (!tail_ready && !(ok = mbar_wait(v_tail, 0, p.wait_ns))) break;
+                    tail_ready = true;
+                    tc_fence_after_sync();
+                    issue_pv(g, i);
+                    if (j + 1 < je_g[g]) {
+                        if (!k_ready && !(ok = mbar_wait(&k_full[(i + 1) & 1], ((i + 1) >> 1) & 1, p.wait_ns)))
+                            break;
+                        k_ready = true;
+                        issue_s(g, i + 1);
+                    }
                 }
-                umma_commit(&pv_done[st]);
+                if (!ok) break;
+                umma_commit(&v_empty[st]);                  // every P V of tile j issued
+                if (next) umma_commit(&k_empty[(i + 1) & 1]);   // every S of tile j+1 issued
             }
-            if (!ok) {
-                abort_now();
-            }
+            if (!ok) abort_now();
             // every MMA this thread issued has completed before TMEM can be released
             umma_commit(drain);
             (void)mbar_wait(drain, 0);
         }
         __syncwarp();
     } else {
-        // ======================================================= softmax warps
-        // Thread (warpgroup g, row r): row r of the tile (TMEM lane r), key columns g*64 .. g*64+63 of
-        // every S tile, and the partial output O_g of those keys (all D columns of row r).
+        // ======================================================= softmax warpgroups
+        // Thread (warpgroup g, row r): row r of query tile g = TMEM lane r, all 128 key columns of S_g,
+        // and row r of O_g.
         const int g = warp >> 2;
         const int r = (warp & 3) * 32 + lane;
-        const int row_in_req = qt * kTile + r;
-        const bool row_valid = row_in_req < L;
-        const int row_pos = min(ctx + row_in_req, kv_len - 1);
-        const int tile_pos0 = ctx + qt * kTile;          // smallest query position in the tile
+        const int cnt = je_g[g] - jb;                    // this tile's key tiles in this CTA
+        const bool row_valid = r < rows_g[g];
+        const int pos_first = ctx + row0 + g * kTile;   // position of the tile's first row
+        const int row_pos = min(pos_first + r, kv_len - 1);
         const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-        const uint32_t o_mine = lane_base + C::kColO + g * D;
+        const uint32_t s_addr = lane_base + C::kColS + g * kTile;
+        const uint32_t o_addr = lane_base + C::kColO + g * D;
         const float qs = p.qscale;
-        float m = -INFINITY, l = 0.f;                    // log2-domain running max and sum of this half
+        float m = -INFINITY, l = 0.f;                    // log2-domain running max and sum of the row
+        // the warp's lanes agree on every wait's outcome, so the .sync.aligned TMEM accesses after it
+        // are never reached by part of a warp
+        auto warp_wait = [&](uint64_t* bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, p.wait_ns));
+        };
         // failure-detection test: the wait runs out and the softmax role stops; the MMA issuer and the
         // producers then run out of their own waits and unwind
-        bool ok = !p.stall || mbar_wait(never, 0, p.wait_ns);
-        for (int j = 0; j < n_tiles && ok; ++j) {
-            if (!(ok = mbar_wait(&s_full[j & 1], (j >> 1) & 1, p.wait_ns))) break;
+        bool ok = !p.stall || warp_wait(never, 0);
+        for (int t = 0; t < cnt && ok; ++t) {            // t: the tile's index among this CTA's tiles
+            const int j = jb + t;
+            if (!(ok = warp_wait(&s_full[g], t & 1))) break;
             tc_fence_after_sync();
             const int key0 = j * kTile;
-            const bool diag = key0 + kTile - 1 > tile_pos0;          // some key of the tile is masked
-            const uint32_t sa = lane_base + C::kColS + (j & 1) * kTile + g * 64;
-            float sv[64];
-            {
-                uint32_t r0[32], r1[32];                  // both loads in flight, one wait
-                tmem_ld_32cols_nowait(sa, r0);
-                tmem_ld_32cols_nowait(sa + 32, r1);
-                tmem_wait_ld();
+            const bool diag = key0 + kTile - 1 > pos_first;     // some key of the tile is masked for some row
+            const int lim = row_pos - key0;                       // columns c <= lim are visible
+            // all 128 scores of the row in registers (one TMEM round trip), masked on diagonal tiles
+            uint32_t sc[4][32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) { sv[i] = __uint_as_float(r0[i]); sv[32 + i] = __uint_as_float(r1[i]); }
-            }
+            for (int c = 0; c < 4; ++c) tmem_ld_32cols_nowait(s_addr + 32 * c, sc[c]);
+            tmem_wait_ld();
             if (diag) {
 #pragma unroll
-                for (int i = 0; i < 64; ++i)
-                    if (key0 + g * 64 + i > row_pos) sv[i] = -INFINITY;
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (32 * c + i > lim) sc[c][i] = __float_as_uint(-INFINITY);
             }
+            // the row max of the raw scores (scale > 0 keeps the order), three operands per instruction
+            auto sf = [&](int k) { return __uint_as_float(sc[k >> 5][k & 31]); };
             float mx8[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) mx8[k] = sv[k];
+            for (int k = 0; k < 8; ++k) mx8[k] = fmax3(sf(k), sf(k + 8), sf(k + 16));
 #pragma unroll
-            for (int i = 8; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
-            // raw scores: scale > 0 keeps the order, so the max is taken before scaling
-            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * qs;
+            for (int k = 24; k < 128; k += 2) mx8[(k >> 1) & 7] = fmax3(mx8[(k >> 1) & 7], sf(k), sf(k + 1));
+            const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                                   fmaxf(mx8[6], mx8[7])) * qs;
             float alpha = 1.f;
-            const bool raise = mx > m + kRescaleLog2;                // false while both are -inf
+            const bool raise = mx > m + kRescaleLog2;            // false while both are -inf
             if (raise) {
-                alpha = exp2f(m - mx);                               // 0 when m is still -inf
+                alpha = exp2f(m - mx);                           // 0 when m is still -inf
                 m = mx;
             }
             const float m_use = m == -INFINITY ? 0.f : m;
-            uint32_t pk[32];
+            // P = 2^(s*qs - m) as fp16 pairs, over the first 64 columns of the S buffer (all of it is in
+            // registers already).  The scaling runs in packed f32x2 arithmetic and every exponential on the
+            // special-function unit: moving a share of them to the FMA pipe measured slower, as this loop is
+            // bound by its dependency latencies rather than by either unit.  The row sum adds the fp16 values
+            // of P that the P V MMA multiplies, so numerator and denominator round alike.
+            const uint64_t qs2 = f32x2_pack(qs, qs), nm2 = f32x2_pack(-m_use, -m_use);
             float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float p0 = exp2f(fmaf(sv[2 * i], qs, -m_use));
-                const float p1 = exp2f(fmaf(sv[2 * i + 1], qs, -m_use));
-                pk[i] = f2_to_h2(p0, p1);
-                rs4[i & 3] = add_h2_f32(rs4[i & 3], pk[i]);   // the fp16 values the P.V MMA adds
+            for (int c = 0; c < 4; ++c) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const uint64_t x = fma_f32x2(
+                        f32x2_pack(__uint_as_float(sc[c][2 * i]), __uint_as_float(sc[c][2 * i + 1])), qs2, nm2);
+                    float x0, x1;
+                    f32x2_unpack(x, x0, x1);
+                    pk[i] = f2_to_h2(exp2f(x0), exp2f(x1));
+                    rs4[i & 3] = add_h2_f32(rs4[i & 3], pk[i]);
+                }
+                tmem_st_16cols_u(s_addr + 16 * c, pk);
             }
             l = fmaf(l, alpha, (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
-            if (j > 0 && __any_sync(0xffffffffu, raise)) {
-                // O_g holds the sum up to tile j-1: wait for that P.V, then rescale this warp's rows
-                if (!(ok = mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, p.wait_ns))) break;
+            if (t > 0 && __any_sync(0xffffffffu, raise)) {
+                // O_g holds the sum up to tile j-1: wait for that P V, then rescale this warp's rows
+                if (!(ok = warp_wait(&pv_done[g], (t - 1) & 1))) break;
                 tc_fence_after_sync();
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     float v[32];
-                    tmem_ld_32cols(o_mine + c * 32, v);
+                    tmem_ld_32cols(o_addr + c * 32, v);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] *= alpha;
-                    tmem_st_32cols(o_mine + c * 32, v);
+                    tmem_st_32cols(o_addr + c * 32, v);
                 }
             }
-            // P (fp16 pairs) over the first half of this thread's S columns, which it has already read;
-            // the P.V of tile j-2, the last reader of this buffer, completed before S(j) did
-            tmem_st_32cols_u(sa, pk);
             tmem_wait_st();
-            if (j == n_tiles - 1 && kv_len < key0 + kTile) {
-                // rows of V past the sequence end may hold anything: zero them before P.V reads them
-                if (!(ok = mbar_wait(&v_full[j & 1], (j >> 1) & 1, p.wait_ns))) break;
-                if (key0 + r >= kv_len) {
-                    uint8_t* vrow = sV + (j & 1) * C::kOpBytes + r * 128;
-#pragma unroll
-                    for (int c = 0; c < C::kChunks; ++c)
-#pragma unroll
-                        for (int u = 0; u < 8 / 2; ++u)
-                            st_shared_u4(vrow + c * C::kChunkBytes + (g * 4 + u) * 16, make_uint4(0, 0, 0, 0));
-                }
-                fence_proxy_async_smem();                     // the zeros reach the tensor core's view
-            }
             tc_fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) mbar_arrive(&p_full[g]);
             if (info[2]) ok = false;
         }
-        // merge the two halves of the row (every softmax thread reaches this barrier)
-        float* red = reinterpret_cast<float*>(smem + C::kOffRed);    // maxes [g][row], then sums [g][row]
-        red[g * 128 + r] = m;
-        red[256 + g * 128 + r] = l;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(sum_bar);
-        if (ok) ok = mbar_wait(sum_bar, 0, p.wait_ns);
-        if (ok) ok = mbar_wait(&pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, p.wait_ns);   // the last P.V has landed
-        if (ok) {
+        if (ok && cnt > 0) ok = warp_wait(&pv_done[g], (cnt - 1) & 1);   // the last P V has landed
+        sm_m = m;
+        sm_l = cnt > 0 ? l : 0.f;
+        sm_cnt = cnt;
+        sm_ok = ok;
+        if (SPLIT == 1 && ok && cnt > 0) {
             tc_fence_after_sync();
-            const float m0 = red[r], m1 = red[128 + r];
-            const float mm = fmaxf(m0, m1);
-            const float c0 = exp2f(m0 - mm), c1 = exp2f(m1 - mm);    // a half that saw no key: 0
-            const float inv = 1.f / (red[256 + r] * c0 + red[384 + r] * c1);
-            const float s0 = c0 * inv, s1 = c1 * inv;
-            constexpr int DH = D / 2;                                // this thread writes columns g*DH ..
-            __half* orow = p.out + (static_cast<int64_t>(q0 + r) * p.H + h) * D + g * DH;
+            const float inv = 1.f / l;
+            __half* orow = p.out + (static_cast<int64_t>(q0 + g * kTile + r) * p.H + h) * D;
 #pragma unroll 1
-            for (int c = 0; c < DH / 32; ++c) {
-                uint32_t a0[32], a1[32];
-                tmem_ld_32cols_nowait(lane_base + C::kColO + g * DH + c * 32, a0);
-                tmem_ld_32cols_nowait(lane_base + C::kColO + D + g * DH + c * 32, a1);
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t a[32];
+                tmem_ld_32cols_nowait(o_addr + c * 32, a);
                 tmem_wait_ld();
                 if (row_valid) {
 #pragma unroll
@@ -441,8 +538,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int i = 8 * q + 2 * e;
-                            ow[e] = f2_to_h2(__uint_as_float(a0[i]) * s0 + __uint_as_float(a1[i]) * s1,
-                                             __uint_as_float(a0[i + 1]) * s0 + __uint_as_float(a1[i + 1]) * s1);
+                            ow[e] = f2_to_h2(__uint_as_float(a[i]) * inv, __uint_as_float(a[i + 1]) * inv);
                         }
                         *reinterpret_cast<uint4*>(orow + c * 32 + 8 * q) = o;
                     }
@@ -450,6 +546,80 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
         }
         if (!ok) abort_now();
+    }
+
+    if constexpr (SPLIT == 2) {
+        // Merge the two halves of every row through distributed shared memory.  After the first cluster
+        // barrier both CTAs are done with their tiles (TMEM holds the final partial O, the K/V stages are
+        // free); CTA c's warpgroup 1-c sends its rows of query tile 1-c (partial O, m, l) into the peer's
+        // K stage area, and after the second barrier CTA c's warpgroup c merges its own rows of tile c
+        // with the peer's and writes them.
+        tc_fence_before_sync();
+        cluster_sync_all();
+        tc_fence_after_sync();
+        float4* rcv_o = reinterpret_cast<float4*>(smem + C::kOffK);      // [D / 4][128] float4
+        float2* rcv_ml = reinterpret_cast<float2*>(smem + C::kOffV);     // [128]
+        const int g = warp >> 2;
+        const int r = (warp & 3) * 32 + lane;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        const uint32_t o_addr = lane_base + C::kColO + g * D;
+        const bool have = sm_ok && sm_cnt > 0;            // warp-uniform
+        if (warp < kSoftmaxWarps && g != crank) {
+            const uint32_t peer = static_cast<uint32_t>(1 - crank);
+            st_cluster_f2(map_to_rank(smem_u32(rcv_ml + r), peer), sm_m, have ? sm_l : 0.f);
+            if (have) {
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t a[32];
+                    tmem_ld_32cols_nowait(o_addr + c * 32, a);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        st_cluster_f4(map_to_rank(smem_u32(rcv_o + (c * 8 + q) * kTile + r), peer),
+                                      __uint_as_float(a[4 * q]), __uint_as_float(a[4 * q + 1]),
+                                      __uint_as_float(a[4 * q + 2]), __uint_as_float(a[4 * q + 3]));
+                }
+            }
+        }
+        cluster_sync_all();
+        if (warp < kSoftmaxWarps && g == crank && rows_g[g] > 0) {
+            const float2 ml1 = rcv_ml[r];
+            const float l0 = have ? sm_l : 0.f, l1 = ml1.y;
+            const float mm = fmaxf(l0 > 0.f ? sm_m : -INFINITY, l1 > 0.f ? ml1.x : -INFINITY);
+            const float w0 = l0 > 0.f ? exp2f(sm_m - mm) : 0.f;
+            const float w1 = l1 > 0.f ? exp2f(ml1.x - mm) : 0.f;
+            const float inv = 1.f / (l0 * w0 + l1 * w1);
+            __half* orow = p.out + (static_cast<int64_t>(q0 + g * kTile + r) * p.H + h) * D;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t a[32];
+                if (have) {
+                    tmem_ld_32cols_nowait(o_addr + c * 32, a);
+                    tmem_wait_ld();
+                }
+                float o[32];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 b = w1 > 0.f ? rcv_o[(c * 8 + q) * kTile + r] : make_float4(0.f, 0.f, 0.f, 0.f);
+                    const float bb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float own = w0 > 0.f ? __uint_as_float(a[4 * q + e]) * w0 : 0.f;
+                        o[4 * q + e] = (own + bb[e] * w1) * inv;
+                    }
+                }
+                if (r < rows_g[g]) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 v;
+                        uint32_t* vw = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) vw[e] = f2_to_h2(o[8 * q + 2 * e], o[8 * q + 2 * e + 1]);
+                        *reinterpret_cast<uint4*>(orow + c * 32 + 8 * q) = v;
+                    }
+                }
+            }
+        }
     }
 
     tc_fence_before_sync();
@@ -460,19 +630,30 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
 }
 
-template <int D>
+template <int D, int SPLIT>
 cudaError_t run_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PrefillParams& p,
-                        dim3 grid, cudaStream_t stream) {
+                        unsigned grid, cudaStream_t stream) {
     using C = PCfg<D>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attr_err = cudaFuncSetAttribute(prefill_kernel<D, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         static_cast<int>(C::kSmemBytes));
     });
     if (attr_err != cudaSuccess) return attr_err;
-    prefill_kernel<D><<<grid, kThreadsP, C::kSmemBytes, stream>>>(tq, tk, tv, p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid * SPLIT);
+    cfg.blockDim = dim3(kThreadsP);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = SPLIT;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = SPLIT > 1 ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, prefill_kernel<D, SPLIT>, tq, tk, tv, p);
 }
 
 }  // namespace
@@ -501,16 +682,31 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream, const char
     p.max_blocks = a.max_blocks;
     p.bs = a.block_size;
     p.num_blocks = a.num_blocks;
-    p.grid_tiles = (a.num_tokens + kTile - 1) / kTile + a.num_reqs;
+    // an upper bound of the query blocks: sum over requests of ceil(L_b / 256)
+    p.grid_blocks = (a.num_tokens + kRowsPerCta - 1) / kRowsPerCta + a.num_reqs;
     p.box_rows = br;
     p.qscale = a.scale * kLog2eP;
     p.err_flag = a.err_flag;
     const uint64_t stall_ns = take_injected_stall(kStallPrefill);
     p.wait_ns = stall_ns ? stall_ns : kWaitLimitNs;
     p.stall = stall_ns != 0;
-    const dim3 grid(p.grid_tiles, a.num_heads);
-    if (a.head_dim == 128) return run_prefill<128>(tq, tk, tv, p, grid, stream);
-    return run_prefill<64>(tq, tk, tv, p, grid, stream);
+    const uint64_t grid = static_cast<uint64_t>(p.grid_blocks) * a.num_heads;
+    if (grid > 0x7fffffffull) {
+        if (why) *why = "too many query blocks x heads for one launch";
+        return cudaErrorInvalidValue;
+    }
+    // Too few (query block, head) pairs to fill the GPU: split every key range over a 2-CTA cluster
+    // (PAGEDKV_PREFILL_SPLIT=0 in the environment turns this off, for comparisons).
+    static const bool split_allowed = [] {
+        const char* e = std::getenv("PAGEDKV_PREFILL_SPLIT");
+        return !(e && e[0] == '0');
+    }();
+    const int64_t pairs = static_cast<int64_t>((a.num_tokens + kRowsPerCta - 1) / kRowsPerCta) * a.num_heads;
+    const bool split = split_allowed && 2 * pairs <= device_sm_count() && 2 * grid <= 0x7fffffffull;
+    const unsigned g = static_cast<unsigned>(grid);
+    if (a.head_dim == 128)
+        return split ? run_prefill<128, 2>(tq, tk, tv, p, g, stream) : run_prefill<128, 1>(tq, tk, tv, p, g, stream);
+    return split ? run_prefill<64, 2>(tq, tk, tv, p, g, stream) : run_prefill<64, 1>(tq, tk, tv, p, g, stream);
 }
 
 }  // namespace pagedkv
