@@ -203,9 +203,10 @@ def _oracle_case(w, budget_tokens):
 # launches of one call.  Workloads without a capture report None, and so must any entry whose kernel has
 # changed since it was taken.
 NCU_TRAFFIC_BYTES = {
-    "b256": {"decode": 2_811_811_000},
-    "b32": {"decode": 276_692_000},
-    "mixed": {"decode": 1_104_481_000, "prefill": 37_940_000},
+    "b256": {"decode": 2_811_942_000},
+    "b32": {"decode": 277_948_000},
+    "mixed": {"decode": 1_104_370_000, "prefill": 38_041_000},
+    "prefill8k": {"prefill": 603_262_000},
 }
 
 
