@@ -691,8 +691,12 @@ def run_serve(args):
     }
     if toks is not None:
         cs = alloc.cache_stats()
+        # every admission (a preempted request is admitted again) either finds a token's K/V in the cache or
+        # prefills it: the hit rate is the cached share of those admitted tokens
+        admitted = st["cached_tokens"] + st["prefill_tokens"]
         line["prefix_cache"] = {"cached_prompt_tokens": st["cached_tokens"], "prompt_tokens": int(prompts.sum()),
-                                "hit_rate": round(st["cached_tokens"] / float(prompts.sum()), 4),
+                                "admitted_prompt_tokens": admitted,
+                                "hit_rate": round(st["cached_tokens"] / float(max(1, admitted)), 4),
                                 "hit_blocks": cs["hit_blocks"], "evictions": cs["evictions"],
                                 "prefix_nodes_at_end": cs["prefix_nodes"], "cached_blocks_at_end": cs["cached_blocks"]}
     print(json.dumps(line), flush=True)
