@@ -91,6 +91,24 @@ def test_prefill_matches_oracle(cuda_ready, H, D, bs, reqs):
     assert diff.max() <= TOL, f"max abs error {diff.max():.3g}"
 
 
+def test_prefill_without_split_matches_oracle(cuda_ready):
+    """The same cases through the one-CTA-per-query-block kernel.  The cases above are small grids, which
+    the launcher runs as 2-CTA clusters that split the key range; PAGEDKV_PREFILL_SPLIT=0 turns the split
+    off (the launcher reads it once per process, hence the child process), so the unsplit kernel gets the
+    ragged tails, head dims, block sizes and multi-request chunks too, and its bounded-wait timeout path."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, PAGEDKV_PREFILL_SPLIT="0")
+    stall = os.path.join(os.path.dirname(__file__), "test_failure_detection_gpu.py")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        f"{__file__}::test_prefill_matches_oracle",
+                        f"{stall}::test_prefill_wait_timeout_is_reported_and_recovered"],
+                       env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
+    assert f"{len(CASES) + 1} passed" in r.stdout, r.stdout[-2000:]
+
+
 def test_mixed_workload_prefill(cuda_ready):
     """The 512-row chunk after 1536 cached tokens of the mixed step, 32 heads x 128."""
     w = si.get("mixed")
