@@ -20,7 +20,8 @@
 //     listed first and the ragged tails last, so the dynamic scheduler hands
 //     out the small items at the end.
 //  2. main kernel (persistent, one CTA per SM, 16 consumer warps + 1
-//     producer warp): the producer pulls items from an atomic counter, reads
+//     producer warp): the producer takes item b first (CTA b), then pulls
+//     items from an atomic counter, reads
 //     the item's block ids (one table entry per lane) and streams 16-token
 //     stages of K and V with one 3-D TMA box each ([16 tokens][HG heads][D],
 //     straight from the paged layout, no gather instructions) into a ring of
@@ -35,7 +36,8 @@
 //     shared-memory slot, so the head merge and the global stores never hold
 //     up the stage ring.
 //  3. combine kernel (one warp per (sequence, head) with several partitions):
-//     m* = max m_i, l* = sum l_i 2^(m_i - m*), o* = sum acc_i 2^(m_i - m*) / l*.
+//     m* = max m_i, l* = sum l_i 2^(m_i - m*), o* = sum acc_i 2^(m_i - m*) / l*;
+//     up to 16 partitions are loaded in one round trip.
 //  Each kernel is launched as a programmatic dependent of the one before: its
 //  CTAs become resident (barriers, TMA descriptors) while the previous kernel
 //  finishes, and wait for it with griddepcontrol before reading its output.
@@ -304,6 +306,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
     pdl_wait();
     constexpr int VEC = D / 32;
     constexpr int kBatch = 8;                   // partitions whose loads are in flight together
+    constexpr int kOneTrip = 16;                // up to this many partitions: all loads in one round trip
     using Vec = typename std::conditional<VEC == 4, float4, float2>::type;
     const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -312,30 +315,53 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(DecodeParams p) {
     const int n = p.n_splits[s];
     if (n <= 1) return;
     const int64_t base = static_cast<int64_t>(s) * p.max_splits * p.H + h;
-    float M = -INFINITY;
-    for (int i = lane; i < n; i += 32) M = fmaxf(M, p.part_ml[base + static_cast<int64_t>(i) * p.H].x);
-    for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float L = 0.f, acc[VEC];
+    float M = -INFINITY, L = 0.f, acc[VEC];
 #pragma unroll
     for (int k = 0; k < VEC; ++k) acc[k] = 0.f;
-    for (int i0 = 0; i0 < n; i0 += kBatch) {
-        // every load of the batch first, then the merge in partition order
-        float2 ml[kBatch];
-        Vec a[kBatch];
+    if (n <= kOneTrip) {
+        // every load at once (one L2 round trip), then the max and the merge in partition order
+        float2 ml[kOneTrip];
+        Vec a[kOneTrip];
 #pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            const int64_t pi = base + static_cast<int64_t>(min(i0 + b, n - 1)) * p.H;
+        for (int b = 0; b < kOneTrip; ++b) {
+            const int64_t pi = base + static_cast<int64_t>(min(b, n - 1)) * p.H;
             ml[b] = p.part_ml[pi];
             a[b] = *reinterpret_cast<const Vec*>(p.part_acc + pi * D + lane * VEC);
         }
 #pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            if (i0 + b >= n) break;
+        for (int b = 0; b < kOneTrip; ++b)
+            if (b < n) M = fmaxf(M, ml[b].x);
+#pragma unroll
+        for (int b = 0; b < kOneTrip; ++b) {
+            if (b >= n) break;
             const float w = exp2f(ml[b].x - M);
             L = fmaf(ml[b].y, w, L);
             const float* av = reinterpret_cast<const float*>(&a[b]);
 #pragma unroll
             for (int k = 0; k < VEC; ++k) acc[k] = fmaf(av[k], w, acc[k]);
+        }
+    } else {
+        for (int i = lane; i < n; i += 32) M = fmaxf(M, p.part_ml[base + static_cast<int64_t>(i) * p.H].x);
+        for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        for (int i0 = 0; i0 < n; i0 += kBatch) {
+            // every load of the batch first, then the merge in partition order
+            float2 ml[kBatch];
+            Vec a[kBatch];
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b) {
+                const int64_t pi = base + static_cast<int64_t>(min(i0 + b, n - 1)) * p.H;
+                ml[b] = p.part_ml[pi];
+                a[b] = *reinterpret_cast<const Vec*>(p.part_acc + pi * D + lane * VEC);
+            }
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b) {
+                if (i0 + b >= n) break;
+                const float w = exp2f(ml[b].x - M);
+                L = fmaf(ml[b].y, w, L);
+                const float* av = reinterpret_cast<const float*>(&a[b]);
+#pragma unroll
+                for (int k = 0; k < VEC; ++k) acc[k] = fmaf(av[k], w, acc[k]);
+            }
         }
     }
     const float r = 1.f / L;
@@ -403,16 +429,16 @@ decode_main_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         uint32_t issued_mask = 0, issued_par = 0;     // per slot: ever issued / parity of its last issue
         bool ok = true;
 
-        int idx = 0;
-        if (lane == 0) idx = atomicAdd(&p.hdr[0], 1);
-        idx = __shfl_sync(0xffffffffu, idx, 0);
+        // CTA b starts with item b (no counter round trip before its first copies); the counter hands out
+        // the items from gridDim.x on
+        const int idx = static_cast<int>(blockIdx.x);
         int4 rec = idx < n_items ? p.items[idx] : make_int4(-1, 0, 0, 0);
         while (rec.x >= 0 && ok) {
             const int seq = rec.x, tok0 = rec.y, ntok_item = rec.z & 1023, hg = rec.z >> 10;
             const int part = rec.w & 0xffff, nsp = rec.w >> 16;
             const int single = nsp == 1;
             int nidx = 0;
-            if (lane == 0) nidx = atomicAdd(&p.hdr[0], 1);       // next item, in flight meanwhile
+            if (lane == 0) nidx = atomicAdd(&p.hdr[0], 1) + static_cast<int>(gridDim.x);   // next item, in flight
             const int blk0 = tok0 / bs;
             const int nblk = (tok0 + ntok_item - 1) / bs - blk0 + 1;
             int bid = 0;
