@@ -163,7 +163,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint64_t* drain = bars + 16;
     uint64_t* never = bars + 17;     // no thread ever arrives on it (failure-detection test)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffSlot);
-    volatile int* info = reinterpret_cast<volatile int*>(smem + C::kOffSlot + 16);   // b, qb, abort
+    // b, qb, abort, and the request's first row, chunk length and cached length
+    volatile int* info = reinterpret_cast<volatile int*>(smem + C::kOffSlot + 16);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const unsigned work = blockIdx.x / SPLIT;           // the two CTAs of a cluster share their work item
@@ -171,31 +172,35 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int h = static_cast<int>(work % static_cast<unsigned>(p.H));
     const int rank = static_cast<int>(work / static_cast<unsigned>(p.H));
 
+    if (warp == kMmaWarp) {                             // TMEM while thread 0 finds the work item
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
     if (threadIdx.x == 0) {
         int g = p.grid_blocks - 1 - rank;        // the latest (heaviest) query blocks go first
-        int bsel = -1, qb = 0;
+        int bsel = -1, qb = 0, s_sel = 0, l_sel = 0, c_sel = 0;
         for (int b = 0; b < p.B; ++b) {
-            const int s0 = p.q_start[b], s1 = p.q_start[b + 1];
+            // the request's cached length is read with its rows, so finding the item is one round trip
+            const int s0 = p.q_start[b], s1 = p.q_start[b + 1], cb = p.ctx_before[b];
             if (s0 < 0 || s1 < s0 || s1 > p.T) {
                 flag_error(p.err_flag, PA_DEVCHK_QUERY_RANGE);
                 bsel = -1;
                 break;
             }
             const int nb = (s1 - s0 + kRowsPerCta - 1) / kRowsPerCta;
-            if (bsel < 0 && g >= 0 && g < nb) { bsel = b; qb = g; }
+            if (bsel < 0 && g >= 0 && g < nb) { bsel = b; qb = g; s_sel = s0; l_sel = s1 - s0; c_sel = cb; }
             g -= nb;
         }
-        if (bsel >= 0) {
-            const int L = p.q_start[bsel + 1] - p.q_start[bsel];
-            const int ctx = p.ctx_before[bsel];
-            if (ctx < 0 || static_cast<int64_t>(ctx) + L > static_cast<int64_t>(p.max_blocks) * p.bs) {
-                flag_error(p.err_flag, PA_DEVCHK_SEQ_LEN);
-                bsel = -1;
-            }
+        if (bsel >= 0 && (c_sel < 0 || static_cast<int64_t>(c_sel) + l_sel > static_cast<int64_t>(p.max_blocks) * p.bs)) {
+            flag_error(p.err_flag, PA_DEVCHK_SEQ_LEN);
+            bsel = -1;
         }
         info[0] = bsel;
         info[1] = qb;
         info[2] = 0;
+        info[3] = s_sel;
+        info[4] = l_sel;
+        info[5] = c_sel;
         mbar_init(q_full, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&k_full[i], kIssueWarps);
@@ -211,13 +216,19 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         mbar_init(never, 1);
         mbar_init_fence();
     }
+    tc_fence_before_sync();
     __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
     const int b = info[0];
-    if (b < 0) return;                                  // uniform: no work for this CTA
+    if (b < 0) {                                        // uniform: no work for this CTA
+        if (warp == kMmaWarp) tmem_dealloc(tmem, C::kTmemCols);
+        return;
+    }
     const int qb = info[1];
-    const int s0 = p.q_start[b];
-    const int L = p.q_start[b + 1] - s0;
-    const int ctx = p.ctx_before[b];
+    const int s0 = info[3];
+    const int L = info[4];
+    const int ctx = info[5];
     const int row0 = qb * kRowsPerCta;                  // first row of Q0 within the request
     const int q0 = s0 + row0;                           // ... within q / out
     // query tile g: its valid rows, the keys its last valid row sees, and the key tiles that covers
@@ -238,15 +249,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     int je_g[kQTiles];                                  // query tile g's key tiles here: [jb, je_g)
 #pragma unroll
     for (int g = 0; g < kQTiles; ++g) je_g[g] = max(jb, min(je, n_g[g]));
-
-    if (warp == kMmaWarp) {
-        tmem_alloc(tmem_slot, C::kTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before_sync();
-    __syncthreads();
-    tc_fence_after_sync();
-    const uint32_t tmem = *tmem_slot;
 
     auto abort_now = [&]() {
         flag_error(p.err_flag, kDevchkTimeout);
