@@ -203,10 +203,10 @@ def _oracle_case(w, budget_tokens):
 # launches of one call.  Workloads without a capture report None, and so must any entry whose kernel has
 # changed since it was taken.
 NCU_TRAFFIC_BYTES = {
-    "b256": {"decode": 2_811_942_000},
-    "b32": {"decode": 277_948_000},
-    "mixed": {"decode": 1_104_370_000, "prefill": 38_041_000},
-    "prefill8k": {"prefill": 603_262_000},
+    "b256": {"decode": 2_812_032_000},
+    "b32": {"decode": 276_752_000},
+    "mixed": {"decode": 1_104_258_000, "prefill": 38_109_000},
+    "prefill8k": {"prefill": 600_975_000},
 }
 
 
