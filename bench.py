@@ -18,6 +18,7 @@ runs it.
 from __future__ import annotations
 
 import argparse
+import datetime
 import json
 import os
 import statistics
@@ -92,23 +93,32 @@ def step_bytes(w, seq_lens, tables_cols, n_step_rows):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clocks and throttle reasons sampled every 50 ms while running; summary() keeps the samples
+    taken between mark_start() and mark_end() (the timed region), or all of them if none can be placed."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_MS = 50
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
+        self.window = [None, None]
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", str(self.PERIOD_MS)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
         return self
+
+    def mark_start(self):
+        self.window[0] = datetime.datetime.now()
+
+    def mark_end(self):
+        self.window[1] = datetime.datetime.now()
 
     def __exit__(self, *exc):
         self.lines = []
@@ -121,33 +131,35 @@ class ClockSampler:
                 out, _ = self.proc.communicate()
             self.lines = [l for l in out.splitlines() if l.strip()]
 
-    def summary(self):
-        sm, mx, reasons = [], None, set()
+    @staticmethod
+    def _parse(line):
+        """(time or None, sm MHz, max MHz, {reason: active}) of one CSV line, or None."""
+        parts = [x.strip() for x in line.split(",")]
+        if len(parts) < 10:
+            return None
+        try:
+            sm, mx = float(parts[2]), float(parts[3])
+        except ValueError:
+            return None
+        try:
+            ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+        except ValueError:
+            ts = None
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
-            parts = [x.strip() for x in l.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return ts, sm, mx, {n: v.lower() == "active" for n, v in zip(names, parts[6:10])}
 
-
-def pool_stats(ds):
-    """Measured internal fragmentation of the pool vs the page's (block_size / 2) / avg_len estimate."""
-    st = ds.alloc.stats()
-    w = ds.workload
-    ctx = int(ds.seq_lens_host.astype(np.int64).sum())
-    return {"block_size": w.block_size, "num_blocks": st["num_blocks"], "used_blocks": st["num_used"],
-            "waste_tokens": st["waste_tokens"], "waste_frac": round(st["waste_tokens"] / max(1, ctx), 5),
-            "page_estimate_frac": round((w.block_size / 2) / (ctx / w.num_seqs), 5) if w.num_seqs and ctx else None}
+    def summary(self):
+        rows = [r for r in (self._parse(l) for l in getattr(self, "lines", [])) if r is not None]
+        lo, hi = self.window
+        if lo is not None and hi is not None:
+            pad = datetime.timedelta(milliseconds=self.PERIOD_MS)
+            inside = [r for r in rows if r[0] is not None and lo - pad <= r[0] <= hi + pad]
+            if inside:
+                rows = inside
+        sm = [r[1] for r in rows]
+        reasons = sorted({n for r in rows for n, on in r[3].items() if on})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": rows[-1][2] if rows else None,
+                "reasons": reasons, "samples": len(sm)}
 
 
 def dist_setup():
@@ -388,6 +400,7 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(device)
+        clk.mark_start()
         t0.record(stream)
         for i in range(args.steps):
             step_events[i].record(stream)
@@ -395,6 +408,7 @@ def run_ours(args):
         step_events[args.steps].record(stream)
         t1.record(stream)
         torch.cuda.synchronize(device)
+        clk.mark_end()
         if world > 1:
             dist.barrier()
     local_ms = t0.elapsed_time(t1)

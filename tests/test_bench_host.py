@@ -118,3 +118,23 @@ def test_reduce_max_sum_two_gloo_ranks():
 
 def test_reduce_is_identity_without_process_group():
     assert bench.reduce_max_sum(3.0, 7.0, torch.device("cpu")) == (3.0, 7.0)
+
+
+def test_clock_summary_keeps_the_timed_window():
+    """Only nvidia-smi samples taken while the timed region ran count; throttle reasons seen outside it do
+    not; lines that cannot be placed in time fall back to all samples."""
+    import datetime
+    c = bench.ClockSampler(0)
+    t = datetime.datetime(2026, 1, 2, 3, 4, 5, 600000)
+    fmt = lambda d: d.strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+    row = lambda d, mhz, cap: (f"{fmt(d)}, 0, {mhz}, 1965, 900.0, 0x0, Not Active, Not Active, Not Active, "
+                               + ("Active" if cap else "Not Active"))
+    c.lines = [row(t - datetime.timedelta(seconds=1), 600, True),          # before: idle, capped
+               row(t, 1965, False), row(t + datetime.timedelta(milliseconds=50), 1900, False),
+               row(t + datetime.timedelta(seconds=2), 700, True),          # after
+               "garbage"]
+    c.window = [t - datetime.timedelta(milliseconds=10), t + datetime.timedelta(milliseconds=60)]
+    assert c.summary() == {"sm_mhz": 1932.5, "sm_max_mhz": 1965.0, "reasons": [], "samples": 2}
+    c.window = [None, None]
+    s = c.summary()
+    assert s["samples"] == 4 and s["reasons"] == ["sw_power_cap"] and s["sm_mhz"] == (700 + 1900) / 2
