@@ -162,6 +162,16 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(sm)}
 
 
+def pool_stats(ds):
+    """Measured internal fragmentation of the pool vs the page's (block_size / 2) / avg_len estimate."""
+    st = ds.alloc.stats()
+    w = ds.workload
+    ctx = int(ds.seq_lens_host.astype(np.int64).sum())
+    return {"block_size": w.block_size, "num_blocks": st["num_blocks"], "used_blocks": st["num_used"],
+            "waste_tokens": st["waste_tokens"], "waste_frac": round(st["waste_tokens"] / max(1, ctx), 5),
+            "page_estimate_frac": round((w.block_size / 2) / (ctx / w.num_seqs), 5) if w.num_seqs and ctx else None}
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

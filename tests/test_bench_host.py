@@ -138,3 +138,21 @@ def test_clock_summary_keeps_the_timed_window():
     c.window = [None, None]
     s = c.summary()
     assert s["samples"] == 4 and s["reasons"] == ["sw_power_cap"] and s["sm_mhz"] == (700 + 1900) / 2
+
+
+def test_pool_stats_against_page_estimate():
+    """kv_pool: measured waste of the allocator beside the page's (bs/2)/avg_len estimate."""
+    import types
+    import paged_kv_cache_411_b200 as pk
+    bs = 16
+    alloc = pk.BlockAllocator(64, bs)
+    lens = np.array([10, 16, 33, 100], np.int32)
+    for r, n in enumerate(lens):
+        assert alloc.allocate(r, int(n)) == pk.PA_OK
+    ds = types.SimpleNamespace(alloc=alloc, seq_lens_host=lens,
+                               workload=types.SimpleNamespace(block_size=bs, num_seqs=len(lens)))
+    st = bench.pool_stats(ds)
+    waste = sum(-(-int(n) // bs) * bs - int(n) for n in lens)          # 6 + 0 + 15 + 12
+    assert st["waste_tokens"] == waste and st["used_blocks"] == sum(-(-int(n) // bs) for n in lens)
+    assert st["waste_frac"] == round(waste / lens.sum(), 5)
+    assert st["page_estimate_frac"] == round((bs / 2) / (lens.sum() / len(lens)), 5)
