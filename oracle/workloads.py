@@ -202,7 +202,7 @@ def build(w: si.Workload, seqs=None) -> OracleStep:
     _check(st)
     return OracleStep(
         workload=w, num_blocks=N, bm=bm, cap_hits=cap_hits, max_blocks=max_blocks,
-        block_tables=np.asarray(tables, dtype=np.int32), seq_lens=np.asarray(lens, dtype=np.int32),
+        block_tables=np.asarray(tables, dtype=np.int32).reshape(-1, max_blocks), seq_lens=np.asarray(lens, dtype=np.int32),
         slot_mapping=np.asarray(step_slots, dtype=np.int64),
         k_step=np.concatenate(k_parts), v_step=np.concatenate(v_parts), q=w.q(),
         k_cache=k_cache, v_cache=v_cache, prefill_q=prefill_q, prefill_table=prefill_table,

@@ -190,7 +190,7 @@ def test_cpp_allocator_error_paths():
     assert st == pk.PA_ERR_NOT_FOUND
 
 
-@pytest.mark.parametrize("name", ["tiny", "b32", "b256", "mixed", "longctx"])
+@pytest.mark.parametrize("name", ["tiny", "b32", "b256", "mixed", "longctx", "prefill8k"])
 def test_workload_replay_matches_oracle(name):
     """Every workload's allocation replay through the C++ allocator is bit-identical to the
     oracle's: pool size, churn cap hits, tables, free list, refcounts, step slot mapping."""
