@@ -74,6 +74,9 @@ CASES = [
     (2, 128, 48, [(47, 81)]),
     (4, 128, 16, [(0, 1), (300, 40), (17, 256), (5, 0), (1000, 130)]),
     (8, 64, 16, [(64, 64), (0, 2), (129, 383)]),
+    # more (query block, head) pairs than SMs: the unsplit kernel, whose CTAs walk several pairs each
+    (16, 128, 16, [(0, 700), (300, 513), (17, 1000), (1000, 130)]),
+    (24, 64, 32, [(64, 300), (0, 1), (129, 900), (5000, 257)]),
 ]
 
 
