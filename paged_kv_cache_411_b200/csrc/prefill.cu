@@ -353,9 +353,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const uint64_t dK = umma_desc_sw128(smem_u32(sK), 16, 1024);
             const uint64_t dV = umma_desc_sw128(smem_u32(sV), C::kChunkBytes, 1024);
             const int n0 = n_g[0], n1 = n_g[1];
-            // An mbarrier answers after ~150 cycles even when its phase is complete, so this thread asks
-            // early (mbar_test_wait) and collects the answers after the MMAs it issues meanwhile; it only
-            // blocks when a phase really is still open.
+            // This thread sets the pace of the tensor core (the MMA queue in front of it is short), so it
+            // waits on each ring barrier once per tile, right before the first MMA that needs it, and a wait
+            // on a phase that has already completed returns in ~15 cycles (mbar_wait tries the phase first).
             // i: the tile's ring position (its index among this CTA's key tiles)
             auto issue_s = [&](int g, int i) {
                 const uint32_t d = tmem + C::kColS + g * kTile;
