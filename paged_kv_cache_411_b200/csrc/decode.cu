@@ -47,7 +47,6 @@
 // nor on which CTA ran which item.
 #include <algorithm>
 #include <type_traits>
-#include <mutex>
 
 #include "device_common.cuh"
 #include "kernels.h"
@@ -690,12 +689,9 @@ template <int D, int HG>
 cudaError_t run_main(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq, const DecodeParams& p,
                      int grid, cudaStream_t stream) {
     using C = Cfg<D, HG>;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(decode_main_kernel<D, HG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        static_cast<int>(C::kSmemBytes));
-    });
+    static std::atomic<uint64_t> smem_set{0};          // devices whose limit is raised
+    const cudaError_t attr_err = ensure_dynamic_smem(reinterpret_cast<const void*>(decode_main_kernel<D, HG>),
+                                                     static_cast<int>(C::kSmemBytes), &smem_set);
     if (attr_err != cudaSuccess) return attr_err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);

@@ -2,6 +2,8 @@
 #pragma once
 
 #include <cuda_runtime.h>
+
+#include <atomic>
 #include <stddef.h>
 #include <stdint.h>
 
@@ -59,6 +61,9 @@ bool encode_tensor_map_3d(void* map_out, const void* base, uint64_t d0, uint64_t
                           uint32_t b2, int swizzle_128b, const char** why);
 
 int32_t device_sm_count();
+// Raises func's dynamic shared-memory limit to `bytes` on the current device, once per device (the setting
+// lives in each device's context); `done` is the caller's per-kernel bitmask of devices already set.
+cudaError_t ensure_dynamic_smem(const void* func, int bytes, std::atomic<uint64_t>* done);
 
 // Failure-detection test hook (pa_debug_inject_stall): the next launch of the given kernel
 // (kStallDecode / kStallPrefill) gets this pipeline-wait limit and makes its consumer role wait on a

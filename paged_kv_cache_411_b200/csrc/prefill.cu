@@ -50,7 +50,6 @@
 // its copies and MMAs drain, frees its TMEM and exits.
 #include <algorithm>
 #include <cstdlib>
-#include <mutex>
 
 #include "device_common.cuh"
 #include "kernels.h"
@@ -636,12 +635,9 @@ template <int D, int SPLIT>
 cudaError_t run_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PrefillParams& p,
                         unsigned grid, cudaStream_t stream) {
     using C = PCfg<D>;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(prefill_kernel<D, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        static_cast<int>(C::kSmemBytes));
-    });
+    static std::atomic<uint64_t> smem_set{0};          // devices whose limit is raised
+    const cudaError_t attr_err = ensure_dynamic_smem(reinterpret_cast<const void*>(prefill_kernel<D, SPLIT>),
+                                                     static_cast<int>(C::kSmemBytes), &smem_set);
     if (attr_err != cudaSuccess) return attr_err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid * SPLIT);

@@ -1,6 +1,7 @@
 // Host runtime helpers of libpagedkv: TMA tensor-map encoding through the
 // driver entry point (so the library needs no link against libcuda) and a
-// per-device SM-count cache used to size persistent grids.
+// per-device SM-count cache used to size persistent grids, and the per-device
+// dynamic shared-memory limit of each kernel.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -62,6 +63,17 @@ int32_t device_sm_count() {
         cache[dev] = n;
     }
     return cache[dev];
+}
+
+cudaError_t ensure_dynamic_smem(const void* func, int bytes, std::atomic<uint64_t>* done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev >= 0 && dev < 64 ? (uint64_t{1} << dev) : 0;
+    if (bit && (done->load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done->fetch_or(bit, std::memory_order_acq_rel);
+    return e;
 }
 
 static std::atomic<uint64_t> g_stall_ns[3];
