@@ -248,6 +248,23 @@ pa_status pa_alloc_cache_stats(const pa_alloc* a, pa_cache_stats_t* out);
  * eviction takes out[0]).  Errors: INVALID_ARG (cap < length; *len_out set). */
 pa_status pa_alloc_evictable_list(const pa_alloc* a, int32_t* out, int32_t cap, int32_t* len_out);
 
+/* Checkpoint of the allocator's host state (no page describes one; [CB-PA] §4.4's swap moves K/V, not the
+ * manager's state): the free-list order, every refcount, each request's block table, length and known
+ * token ids, the prefix trie, the cached blocks, the LRU order and the counters, as a versioned
+ * little-endian byte string.  Maps are written in key order, so equal states give equal bytes, and the
+ * bytes can be compared to diff two allocators.  With buf NULL only *size (the bytes needed) is set and
+ * PA_OK returned; otherwise capacity must be >= that size (INVALID_ARG if not, nothing written).  The K/V
+ * pool contents are not part of it (they are the caller's device memory).
+ * Errors: INVALID_ARG. */
+pa_status pa_alloc_serialize(const pa_alloc* a, uint8_t* buf, size_t capacity, size_t* size);
+
+/* Creates an allocator holding a state written by pa_alloc_serialize (resume).  The bytes are checked
+ * before use: format and version, every count against the buffer's length, every block id in the pool,
+ * no block listed twice in the free list or the LRU, table lengths against request lengths, trie parents
+ * present.  On any error nothing is created and *out is NULL.
+ * Errors: INVALID_ARG, OOM. */
+pa_status pa_alloc_deserialize(const uint8_t* buf, size_t size, pa_alloc** out);
+
 /* ---- swap between the GPU pool and a host pool ([CB-PA] §4.4 Swap: CPU
  * offload, one block manager per pool; §5.4 preemption by swapping) ---------
  *

@@ -12,7 +12,7 @@ used for device memory and streams, every computation runs in the library.
 from __future__ import annotations
 
 import ctypes
-from ctypes import POINTER, byref, c_int32, c_int64, c_void_p
+from ctypes import POINTER, byref, c_int32, c_int64, c_size_t, c_void_p
 
 import numpy as np
 
@@ -57,6 +57,26 @@ class BlockAllocator:
         if self._h:
             lib().pa_alloc_destroy(self._h)
             self._h = c_void_p()
+
+    def serialize(self) -> bytes:
+        """pa_alloc_serialize: the allocator's whole host state as bytes (equal states, equal bytes)."""
+        n = c_size_t(0)
+        check(lib().pa_alloc_serialize(self._h, None, 0, byref(n)))
+        buf = (ctypes.c_uint8 * max(n.value, 1))()
+        check(lib().pa_alloc_serialize(self._h, ctypes.cast(buf, c_void_p), n.value, byref(n)))
+        return bytes(buf)[:n.value]
+
+    @classmethod
+    def deserialize(cls, data: bytes) -> "BlockAllocator":
+        """pa_alloc_deserialize: a new allocator holding a state written by serialize() (raises on bad bytes)."""
+        raw = (ctypes.c_uint8 * max(len(data), 1)).from_buffer_copy(data if data else b"\0")
+        h = c_void_p()
+        check(lib().pa_alloc_deserialize(ctypes.cast(raw, c_void_p), len(data), byref(h)))
+        obj = cls.__new__(cls)
+        obj._h = h
+        hdr = np.frombuffer(bytes(data[8:16]), dtype=np.int32)
+        obj.num_blocks, obj.block_size = int(hdr[0]), int(hdr[1])
+        return obj
 
     def __del__(self):
         try:

@@ -126,6 +126,8 @@ SIGNATURES = {
     "pa_alloc_begin_cached": (c_int32, [_P, c_int64, _I32P, c_int32, _I32P]),
     "pa_alloc_extend_tokens": (c_int32, [_P, c_int64, _I32P, c_int32]),
     "pa_alloc_evictable_list": (c_int32, [_P, _I32P, c_int32, _I32P]),
+    "pa_alloc_serialize": (c_int32, [_P, _P, c_size_t, POINTER(c_size_t)]),
+    "pa_alloc_deserialize": (c_int32, [_P, c_size_t, POINTER(c_void_p)]),
     "pa_swap_blocks": (c_int32, [_P, _P, _P, _P, _I64P, c_int32, c_int64, c_int32, c_int32, _P]),
     "pa_alloc_swap_out": (c_int32, [_P, _P, c_int64, _P, _P, _P, _P, c_int64, _P]),
     "pa_alloc_swap_in": (c_int32, [_P, _P, c_int64, _P, _P, _P, _P, c_int64, _P]),

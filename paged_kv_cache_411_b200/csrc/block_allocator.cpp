@@ -553,3 +553,205 @@ pa_status pa_alloc_evictable_list(const pa_alloc* a, int32_t* out, int32_t cap, 
 }
 
 }  // extern "C"
+
+// ---- checkpoint / resume of the host state ----------------------------------------------------------
+// Format (little-endian, version 1): "PKVA", u32 version, i32 num_blocks, i32 block_size, i64 oom_count,
+// i64 hit_blocks, i64 evictions, i64 next_node; u64 n, i32 free_list[n] (bottom of the stack first);
+// i32 refcount[num_blocks]; u64 n_requests, then per request in increasing id: i64 id, i32 len, u8 tracked,
+// i64 last_node, u64 n, i32 table[n], u64 m, i32 tokens[m]; u64 n_nodes, then per trie node in increasing
+// id: i64 node, i64 parent, i32 children, i32 cached block (-1: none), i32 tokens[block_size]; u64 n,
+// i32 lru[n] (least recently used first).  Maps are written in key order, so equal states give equal bytes.
+namespace {
+
+constexpr uint32_t kStateVersion = 1;
+
+struct Writer {
+    uint8_t* buf;
+    size_t cap, n = 0;
+    template <typename T>
+    void put(T v) {
+        if (buf && n + sizeof(T) <= cap) std::memcpy(buf + n, &v, sizeof(T));
+        n += sizeof(T);
+    }
+    void put_i32s(const int32_t* v, size_t count) {
+        put<uint64_t>(count);
+        for (size_t i = 0; i < count; ++i) put<int32_t>(v[i]);
+    }
+};
+
+struct Reader {
+    const uint8_t* buf;
+    size_t size, n = 0;
+    bool ok = true;
+    template <typename T>
+    T get() {
+        T v{};
+        if (!ok || n + sizeof(T) > size) {
+            ok = false;
+            return v;
+        }
+        std::memcpy(&v, buf + n, sizeof(T));
+        n += sizeof(T);
+        return v;
+    }
+    // a count of int32 entries that must still fit in the buffer
+    uint64_t count() {
+        const uint64_t c = get<uint64_t>();
+        if (ok && c > (size - n) / sizeof(int32_t)) ok = false;
+        return ok ? c : 0;
+    }
+};
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_alloc_serialize(const pa_alloc* a, uint8_t* buf, size_t capacity, size_t* size) {
+    if (!a || !size) return fail(PA_ERR_INVALID_ARG, "pa_alloc_serialize: NULL argument");
+    auto write = [&](Writer& w) {
+        w.put<uint32_t>(0x41564B50u);   // "PKVA"
+        w.put<uint32_t>(kStateVersion);
+        w.put<int32_t>(a->num_blocks);
+        w.put<int32_t>(a->block_size);
+        w.put<int64_t>(a->oom_count);
+        w.put<int64_t>(a->hit_blocks);
+        w.put<int64_t>(a->evictions);
+        w.put<int64_t>(a->next_node);
+        w.put_i32s(a->free_list.data(), a->free_list.size());
+        for (int32_t b = 0; b < a->num_blocks; ++b) w.put<int32_t>(a->refcount[b]);
+        std::vector<int64_t> ids;
+        for (const auto& kv : a->reqs) ids.push_back(kv.first);
+        std::sort(ids.begin(), ids.end());
+        w.put<uint64_t>(ids.size());
+        for (int64_t id : ids) {
+            const auto& r = a->reqs.at(id);
+            w.put<int64_t>(id);
+            w.put<int32_t>(r.len);
+            w.put<uint8_t>(r.tracked ? 1 : 0);
+            w.put<int64_t>(r.last_node);
+            w.put_i32s(r.table.data(), r.table.size());
+            w.put_i32s(r.tokens.data(), r.tokens.size());
+        }
+        std::vector<int64_t> nodes;
+        for (const auto& kv : a->node_key) nodes.push_back(kv.first);
+        std::sort(nodes.begin(), nodes.end());
+        w.put<uint64_t>(nodes.size());
+        for (int64_t node : nodes) {
+            const PrefixKey& k = a->node_key.at(node);
+            auto ch = a->children.find(node);
+            auto c = a->cache.find(node);
+            w.put<int64_t>(node);
+            w.put<int64_t>(k.parent);
+            w.put<int32_t>(ch == a->children.end() ? 0 : ch->second);
+            w.put<int32_t>(c == a->cache.end() ? -1 : c->second);
+            for (int32_t t : k.tokens) w.put<int32_t>(t);
+        }
+        w.put<uint64_t>(a->lru.size());
+        for (int32_t b : a->lru) w.put<int32_t>(b);
+    };
+    Writer probe{nullptr, 0};
+    write(probe);
+    *size = probe.n;
+    if (!buf) return PA_OK;                                   // size query
+    if (capacity < probe.n)
+        return fail(PA_ERR_INVALID_ARG, "pa_alloc_serialize: capacity %zu < %zu bytes", capacity, probe.n);
+    Writer w{buf, capacity};
+    write(w);
+    return PA_OK;
+}
+
+pa_status pa_alloc_deserialize(const uint8_t* buf, size_t size, pa_alloc** out) {
+    if (!out) return fail(PA_ERR_INVALID_ARG, "pa_alloc_deserialize: out is NULL");
+    *out = nullptr;
+    if (!buf) return fail(PA_ERR_INVALID_ARG, "pa_alloc_deserialize: NULL buffer");
+    Reader r{buf, size};
+    if (r.get<uint32_t>() != 0x41564B50u || r.get<uint32_t>() != kStateVersion || !r.ok)
+        return fail(PA_ERR_INVALID_ARG, "pa_alloc_deserialize: not an allocator state of version %u", kStateVersion);
+    const int32_t nb = r.get<int32_t>(), bs = r.get<int32_t>();
+    // every count below must be backed by bytes of the buffer before anything is sized from it
+    if (!r.ok || nb < 0 || bs <= 0 || static_cast<uint64_t>(nb) > (size - r.n) / sizeof(int32_t) ||
+        static_cast<uint64_t>(bs) > (size - r.n) / sizeof(int32_t))
+        return fail(PA_ERR_INVALID_ARG, "pa_alloc_deserialize: bad pool shape");
+    pa_alloc* a = nullptr;
+    if (pa_alloc_create(nb, bs, nullptr, &a) != PA_OK) return PA_ERR_OOM;
+    auto bad = [&](const char* what) {
+        delete a;
+        return fail(PA_ERR_INVALID_ARG, "pa_alloc_deserialize: %s", what);
+    };
+    auto block_ok = [&](int64_t b) { return b >= 0 && b < nb; };
+    a->oom_count = r.get<int64_t>();
+    a->hit_blocks = r.get<int64_t>();
+    a->evictions = r.get<int64_t>();
+    a->next_node = r.get<int64_t>();
+    const uint64_t nf = r.count();
+    if (!r.ok || nf > static_cast<uint64_t>(nb)) return bad("free list");
+    a->free_list.assign(nf, 0);
+    std::vector<char> seen(nb, 0);
+    for (uint64_t i = 0; i < nf; ++i) {
+        const int32_t b = r.get<int32_t>();
+        if (!r.ok || !block_ok(b) || seen[b]) return bad("free list entry");
+        seen[b] = 1;
+        a->free_list[i] = b;
+    }
+    for (int32_t b = 0; b < nb; ++b) {
+        a->refcount[b] = r.get<int32_t>();
+        if (!r.ok || a->refcount[b] < 0) return bad("refcount");
+    }
+    const uint64_t nr = r.get<uint64_t>();
+    for (uint64_t i = 0; r.ok && i < nr; ++i) {
+        const int64_t id = r.get<int64_t>();
+        pa_alloc::Request q;
+        q.len = r.get<int32_t>();
+        q.tracked = r.get<uint8_t>() != 0;
+        q.last_node = r.get<int64_t>();
+        const uint64_t nt = r.count();
+        for (uint64_t k = 0; r.ok && k < nt; ++k) {
+            const int32_t b = r.get<int32_t>();
+            if (!block_ok(b)) return bad("table entry");
+            q.table.push_back(b);
+        }
+        const uint64_t nk = r.count();
+        for (uint64_t k = 0; r.ok && k < nk; ++k) q.tokens.push_back(r.get<int32_t>());
+        if (!r.ok || q.len < 0 || static_cast<int64_t>(q.table.size()) != a->blocks_for(q.len) ||
+            a->reqs.count(id))
+            return bad("request");
+        a->reqs.emplace(id, std::move(q));
+    }
+    const uint64_t nn = r.get<uint64_t>();
+    for (uint64_t i = 0; r.ok && i < nn; ++i) {
+        const int64_t node = r.get<int64_t>(), parent = r.get<int64_t>();
+        const int32_t nch = r.get<int32_t>(), blk = r.get<int32_t>();
+        if (!r.ok || static_cast<uint64_t>(bs) > (size - r.n) / sizeof(int32_t)) return bad("trie node");
+        PrefixKey k{parent, std::vector<int32_t>(bs)};
+        for (int32_t t = 0; t < bs; ++t) k.tokens[t] = r.get<int32_t>();
+        if (!r.ok || node < 0 || node >= a->next_node || nch < 0 || (blk != -1 && !block_ok(blk)) ||
+            a->node_key.count(node) || a->trie.count(k))
+            return bad("trie node");
+        a->node_key.emplace(node, k);
+        a->trie.emplace(std::move(k), node);
+        a->children[node] = nch;
+        if (blk >= 0) {
+            if (a->block_node[blk] != -1) return bad("block cached twice");
+            a->cache.emplace(node, blk);
+            a->block_node[blk] = node;
+        }
+    }
+    // every parent and every request's last registered node is a node of the trie (or the root)
+    for (const auto& kv : a->node_key)
+        if (kv.second.parent != -1 && !a->node_key.count(kv.second.parent)) return bad("trie parent");
+    for (const auto& kv : a->reqs)
+        if (kv.second.last_node != -1 && !a->node_key.count(kv.second.last_node)) return bad("request node");
+    const uint64_t nl = r.count();
+    for (uint64_t i = 0; r.ok && i < nl; ++i) {
+        const int32_t b = r.get<int32_t>();
+        if (!block_ok(b) || a->in_lru[b] || a->block_node[b] < 0 || a->refcount[b] != 0) return bad("LRU entry");
+        a->lru.push_back(b);
+        a->lru_pos[b] = std::prev(a->lru.end());
+        a->in_lru[b] = 1;
+    }
+    if (!r.ok || r.n != size) return bad("length");
+    *out = a;
+    return PA_OK;
+}
+
+}  // extern "C"
