@@ -33,11 +33,12 @@ SOURCES = [
     "decode.cu",
     "decode_noalloc.cu",
     "prefill.cu",
+    "prefill_q128.cu",
 ]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 # Per-file extra flags: the prefill softmax evaluates 16k exp2 per 128x128 tile, so it uses the
 # hardware exp2 (fast-math); its results are checked against the float64 oracle like the rest.
-EXTRA = {"prefill.cu": ["--use_fast_math"]}
+EXTRA = {"prefill.cu": ["--use_fast_math"], "prefill_q128.cu": ["--use_fast_math"]}
 
 
 def nvcc() -> str:

@@ -53,6 +53,10 @@ struct PrefillArgs {
 
 bool prefill_supported(int32_t num_heads, int32_t head_dim, int32_t block_size);
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream, const char** why);
+// The one-query-tile prefill kernel (prefill_q128.cu) that launch_prefill uses for small launches;
+// wait_ns and stall are the launch's pipeline-wait limit and failure-detection test switch.
+cudaError_t launch_prefill_q128(const PrefillArgs& a, uint64_t wait_ns, bool stall, cudaStream_t stream,
+                                const char** why);
 
 // Tensor-map encoding through the driver entry point (no libcuda link).
 // Returns false and sets *why on failure.

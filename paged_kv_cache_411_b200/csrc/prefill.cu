@@ -41,11 +41,8 @@
 //     MMA adds.  After the last tile each thread normalises its row of O_g and
 //     stores it as fp16.
 // When a launch has too few (256-row query block, head) pairs to fill the GPU
-// (a short chunk after a long cached prefix), it runs in clusters of two CTAs
-// per pair instead: each CTA takes half of the key tiles, and the two partial
-// results of every row, (O, m, l), are merged with the log-sum-exp rule
-// through distributed shared memory at the end (no workspace, no second
-// launch); CTA c of the cluster finalises query tile c.
+// (a short chunk after a long cached prefix), the launcher runs the
+// one-query-tile kernel of prefill_q128.cu instead, with twice as many CTAs.
 // Every wait is bounded; on a timeout the CTA records PA_DEVCHK_TIMEOUT, lets
 // its copies and MMAs drain, frees its TMEM and exits.
 #include <algorithm>
@@ -110,36 +107,7 @@ __device__ __forceinline__ void st_shared_zero16(uint32_t addr) {
     asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0) : "memory");
 }
 
-// ---- thread-block cluster (split key range): the two CTAs of a cluster exchange partial rows
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-// Every thread of both CTAs arrives (release) and waits (acquire): shared-memory writes made before it,
-// local or remote, are visible after it.
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// The shared::cluster address of this CTA's shared-memory address `a` in the cluster's CTA `rank`.
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t a, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ void st_cluster_f4(uint32_t addr, float a, float b, float c, float d) {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-                 : "memory");
-}
-__device__ __forceinline__ void st_cluster_f2(uint32_t addr, float a, float b) {
-    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
-}
-
-// SPLIT == 2: the kernel is launched in clusters of two CTAs that share one (query block, head); CTA c of
-// the cluster runs key tiles [jb, je) (the first or the second half of the key range), and the two partial
-// results of every row are merged through distributed shared memory at the end, CTA c finalising query
-// tile c.  Used when the launch has too few (query block, head) pairs to fill the GPU.
-template <int D, int SPLIT>
+template <int D>
 __global__ void __launch_bounds__(kThreadsP, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, PrefillParams p) {
@@ -166,8 +134,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     volatile int* info = reinterpret_cast<volatile int*>(smem + C::kOffSlot + 16);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const unsigned work = blockIdx.x / SPLIT;           // the two CTAs of a cluster share their work item
-    const int crank = SPLIT == 2 ? static_cast<int>(cluster_ctarank()) : 0;
+    const unsigned work = blockIdx.x;                   // the (query block, head) pair of this CTA
     const int h = static_cast<int>(work % static_cast<unsigned>(p.H));
     const int rank = static_cast<int>(work / static_cast<unsigned>(p.H));
 
@@ -240,12 +207,10 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     const int kv_len = max(kvl_g[0], kvl_g[1]);
     const int n_tiles = max(n_g[0], n_g[1]);            // >= 1: Q0 always has a valid row
-    // this CTA's key tiles [jb, je): all of them, or one half of them in a split cluster
-    const int half = (n_tiles + 1) / 2;
-    const int jb = (SPLIT == 2 && crank == 1) ? half : 0;
-    const int je = (SPLIT == 2 && crank == 0) ? half : n_tiles;
-    const int n_loc = je - jb;                          // may be 0 (the second CTA of a one-tile block)
-    int je_g[kQTiles];                                  // query tile g's key tiles here: [jb, je_g)
+    // this CTA's key tiles [jb, je) and query tile g's share of them [jb, je_g)
+    const int jb = 0, je = n_tiles;
+    const int n_loc = je - jb;
+    int je_g[kQTiles];
 #pragma unroll
     for (int g = 0; g < kQTiles; ++g) je_g[g] = max(jb, min(je, n_g[g]));
 
@@ -253,11 +218,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         flag_error(p.err_flag, kDevchkTimeout);
         info[2] = 1;
     };
-    // a softmax thread's partial result for the split merge: running max, sum, its tile count, no timeout
-    float sm_m = -INFINITY, sm_l = 0.f;
-    int sm_cnt = 0;
-    bool sm_ok = false;
-
     if (warp >= kFirstKWarp && warp < kMmaWarp) {
         // ======================================================= TMA producers (K warps, V warps)
         // A 128-key tile is one box per (physical block, 64-dim chunk).  The boxes of a tile are dealt
@@ -518,11 +478,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (info[2]) ok = false;
         }
         if (ok && cnt > 0) ok = warp_wait(&pv_done[g], (cnt - 1) & 1);   // the last P V has landed
-        sm_m = m;
-        sm_l = cnt > 0 ? l : 0.f;
-        sm_cnt = cnt;
-        sm_ok = ok;
-        if (SPLIT == 1 && ok && cnt > 0) {
+        if (ok && cnt > 0) {
             tc_fence_after_sync();
             const float inv = 1.f / l;
             __half* orow = p.out + (static_cast<int64_t>(q0 + g * kTile + r) * p.H + h) * D;
@@ -549,80 +505,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (!ok) abort_now();
     }
 
-    if constexpr (SPLIT == 2) {
-        // Merge the two halves of every row through distributed shared memory.  After the first cluster
-        // barrier both CTAs are done with their tiles (TMEM holds the final partial O, the K/V stages are
-        // free); CTA c's warpgroup 1-c sends its rows of query tile 1-c (partial O, m, l) into the peer's
-        // K stage area, and after the second barrier CTA c's warpgroup c merges its own rows of tile c
-        // with the peer's and writes them.
-        tc_fence_before_sync();
-        cluster_sync_all();
-        tc_fence_after_sync();
-        float4* rcv_o = reinterpret_cast<float4*>(smem + C::kOffK);      // [D / 4][128] float4
-        float2* rcv_ml = reinterpret_cast<float2*>(smem + C::kOffV);     // [128]
-        const int g = warp >> 2;
-        const int r = (warp & 3) * 32 + lane;
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-        const uint32_t o_addr = lane_base + C::kColO + g * D;
-        const bool have = sm_ok && sm_cnt > 0;            // warp-uniform
-        if (warp < kSoftmaxWarps && g != crank) {
-            const uint32_t peer = static_cast<uint32_t>(1 - crank);
-            st_cluster_f2(map_to_rank(smem_u32(rcv_ml + r), peer), sm_m, have ? sm_l : 0.f);
-            if (have) {
-#pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t a[32];
-                    tmem_ld_32cols_nowait(o_addr + c * 32, a);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        st_cluster_f4(map_to_rank(smem_u32(rcv_o + (c * 8 + q) * kTile + r), peer),
-                                      __uint_as_float(a[4 * q]), __uint_as_float(a[4 * q + 1]),
-                                      __uint_as_float(a[4 * q + 2]), __uint_as_float(a[4 * q + 3]));
-                }
-            }
-        }
-        cluster_sync_all();
-        if (warp < kSoftmaxWarps && g == crank && rows_g[g] > 0) {
-            const float2 ml1 = rcv_ml[r];
-            const float l0 = have ? sm_l : 0.f, l1 = ml1.y;
-            const float mm = fmaxf(l0 > 0.f ? sm_m : -INFINITY, l1 > 0.f ? ml1.x : -INFINITY);
-            const float w0 = l0 > 0.f ? exp2f(sm_m - mm) : 0.f;
-            const float w1 = l1 > 0.f ? exp2f(ml1.x - mm) : 0.f;
-            const float inv = 1.f / (l0 * w0 + l1 * w1);
-            __half* orow = p.out + (static_cast<int64_t>(q0 + g * kTile + r) * p.H + h) * D;
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t a[32];
-                if (have) {
-                    tmem_ld_32cols_nowait(o_addr + c * 32, a);
-                    tmem_wait_ld();
-                }
-                float o[32];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 b = w1 > 0.f ? rcv_o[(c * 8 + q) * kTile + r] : make_float4(0.f, 0.f, 0.f, 0.f);
-                    const float bb[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float own = w0 > 0.f ? __uint_as_float(a[4 * q + e]) * w0 : 0.f;
-                        o[4 * q + e] = (own + bb[e] * w1) * inv;
-                    }
-                }
-                if (r < rows_g[g]) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint4 v;
-                        uint32_t* vw = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) vw[e] = f2_to_h2(o[8 * q + 2 * e], o[8 * q + 2 * e + 1]);
-                        *reinterpret_cast<uint4*>(orow + c * 32 + 8 * q) = v;
-                    }
-                }
-            }
-        }
-    }
-
     tc_fence_before_sync();
     __syncthreads();
     if (warp == kMmaWarp) {
@@ -631,27 +513,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
 }
 
-template <int D, int SPLIT>
+template <int D>
 cudaError_t run_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const PrefillParams& p,
                         unsigned grid, cudaStream_t stream) {
     using C = PCfg<D>;
     static std::atomic<uint64_t> smem_set{0};          // devices whose limit is raised
-    const cudaError_t attr_err = ensure_dynamic_smem(reinterpret_cast<const void*>(prefill_kernel<D, SPLIT>),
+    const cudaError_t attr_err = ensure_dynamic_smem(reinterpret_cast<const void*>(prefill_kernel<D>),
                                                      static_cast<int>(C::kSmemBytes), &smem_set);
     if (attr_err != cudaSuccess) return attr_err;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid * SPLIT);
-    cfg.blockDim = dim3(kThreadsP);
-    cfg.dynamicSmemBytes = C::kSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = SPLIT;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = SPLIT > 1 ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, prefill_kernel<D, SPLIT>, tq, tk, tv, p);
+    prefill_kernel<D><<<grid, kThreadsP, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -661,6 +532,17 @@ bool prefill_supported(int32_t H, int32_t D, int32_t bs) {
 }
 
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream, const char** why) {
+    const uint64_t stall_ns = take_injected_stall(kStallPrefill);
+    const uint64_t wait_ns = stall_ns ? stall_ns : kWaitLimitNs;
+    // Too few (256-row query block, head) pairs to fill the GPU: the one-query-tile kernel, twice the CTAs
+    // (PAGEDKV_PREFILL_SPLIT=0 in the environment keeps this kernel, for comparisons and tests).
+    static const bool small_allowed = [] {
+        const char* e = std::getenv("PAGEDKV_PREFILL_SPLIT");
+        return !(e && e[0] == '0');
+    }();
+    const int64_t pairs = static_cast<int64_t>((a.num_tokens + kRowsPerCta - 1) / kRowsPerCta) * a.num_heads;
+    if (small_allowed && 2 * pairs <= device_sm_count()) return launch_prefill_q128(a, wait_ns, stall_ns != 0, stream, why);
+
     const int br = std::min(kTile, a.block_size & -a.block_size);    // largest power of two dividing bs, <= 128
     const uint64_t s1 = static_cast<uint64_t>(a.head_dim) * 2, s2 = s1 * a.num_heads;
     const uint64_t rows = static_cast<uint64_t>(a.num_blocks) * a.block_size;
@@ -685,26 +567,15 @@ cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream, const char
     p.box_rows = br;
     p.qscale = a.scale * kLog2eP;
     p.err_flag = a.err_flag;
-    const uint64_t stall_ns = take_injected_stall(kStallPrefill);
-    p.wait_ns = stall_ns ? stall_ns : kWaitLimitNs;
+    p.wait_ns = wait_ns;
     p.stall = stall_ns != 0;
     const uint64_t grid = static_cast<uint64_t>(p.grid_blocks) * a.num_heads;
     if (grid > 0x7fffffffull) {
         if (why) *why = "too many query blocks x heads for one launch";
         return cudaErrorInvalidValue;
     }
-    // Too few (query block, head) pairs to fill the GPU: split every key range over a 2-CTA cluster
-    // (PAGEDKV_PREFILL_SPLIT=0 in the environment turns this off, for comparisons).
-    static const bool split_allowed = [] {
-        const char* e = std::getenv("PAGEDKV_PREFILL_SPLIT");
-        return !(e && e[0] == '0');
-    }();
-    const int64_t pairs = static_cast<int64_t>((a.num_tokens + kRowsPerCta - 1) / kRowsPerCta) * a.num_heads;
-    const bool split = split_allowed && 2 * pairs <= device_sm_count() && 2 * grid <= 0x7fffffffull;
     const unsigned g = static_cast<unsigned>(grid);
-    if (a.head_dim == 128)
-        return split ? run_prefill<128, 2>(tq, tk, tv, p, g, stream) : run_prefill<128, 1>(tq, tk, tv, p, g, stream);
-    return split ? run_prefill<64, 2>(tq, tk, tv, p, g, stream) : run_prefill<64, 1>(tq, tk, tv, p, g, stream);
+    return a.head_dim == 128 ? run_prefill<128>(tq, tk, tv, p, g, stream) : run_prefill<64>(tq, tk, tv, p, g, stream);
 }
 
 }  // namespace pagedkv

@@ -95,10 +95,10 @@ def test_prefill_matches_oracle(cuda_ready, H, D, bs, reqs):
 
 
 def test_prefill_without_split_matches_oracle(cuda_ready):
-    """The same cases through the one-CTA-per-query-block kernel.  The cases above are small grids, which
-    the launcher runs as 2-CTA clusters that split the key range; PAGEDKV_PREFILL_SPLIT=0 turns the split
-    off (the launcher reads it once per process, hence the child process), so the unsplit kernel gets the
-    ragged tails, head dims, block sizes and multi-request chunks too, and its bounded-wait timeout path."""
+    """The same cases through the two-query-tile kernel.  The cases above are small launches, which the
+    launcher gives to the one-query-tile kernel; PAGEDKV_PREFILL_SPLIT=0 turns that off (the launcher reads
+    it once per process, hence the child process), so the two-query-tile kernel gets the ragged tails, head
+    dims, block sizes and multi-request chunks too, and its bounded-wait timeout path."""
     import os
     import subprocess
     import sys
