@@ -355,14 +355,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 for (int i = 0; i < 64; ++i)
                     if (key0 + g * 64 + i > row_pos) sv[i] = -INFINITY;
             }
+            // raw scores: scale > 0 keeps the order, so the max is taken before scaling (three operands per
+            // instruction)
             float mx8[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) mx8[k] = sv[k];
+            for (int k = 0; k < 8; ++k) mx8[k] = fmax3(sv[k], sv[k + 8], sv[k + 16]);
 #pragma unroll
-            for (int i = 8; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
-            // raw scores: scale > 0 keeps the order, so the max is taken before scaling
-            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * qs;
+            for (int i = 24; i < 64; i += 2) mx8[(i >> 1) & 7] = fmax3(mx8[(i >> 1) & 7], sv[i], sv[i + 1]);
+            const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                                   fmaxf(mx8[6], mx8[7])) * qs;
             float alpha = 1.f;
             const bool raise = mx > m + kRescaleLog2;                // false while both are -inf
             if (raise) {
@@ -372,11 +373,12 @@ prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const float m_use = m == -INFINITY ? 0.f : m;
             uint32_t pk[32];
             float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+            const uint64_t qs2 = f32x2_pack(qs, qs), nm2 = f32x2_pack(-m_use, -m_use);
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float p0 = exp2f(fmaf(sv[2 * i], qs, -m_use));
-                const float p1 = exp2f(fmaf(sv[2 * i + 1], qs, -m_use));
-                pk[i] = f2_to_h2(p0, p1);
+                float x0, x1;                             // the scaling in packed f32x2 arithmetic
+                f32x2_unpack(fma_f32x2(f32x2_pack(sv[2 * i], sv[2 * i + 1]), qs2, nm2), x0, x1);
+                pk[i] = f2_to_h2(exp2f(x0), exp2f(x1));
                 rs4[i & 3] = add_h2_f32(rs4[i & 3], pk[i]);   // the fp16 values the P.V MMA adds
             }
             l = fmaf(l, alpha, (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
