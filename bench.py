@@ -227,7 +227,7 @@ def _oracle_case(w, budget_tokens):
 NCU_TRAFFIC_BYTES = {
     "b256": {"decode": 2_812_032_000},
     "b32": {"decode": 276_752_000},
-    "mixed": {"decode": 1_104_424_000, "prefill": 37_968_000},
+    "mixed": {"decode": 1_104_322_000, "prefill": 37_870_000},
     "prefill8k": {"prefill": 600_975_000},
 }
 
