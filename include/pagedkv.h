@@ -261,7 +261,10 @@ pa_status pa_alloc_serialize(const pa_alloc* a, uint8_t* buf, size_t capacity, s
 /* Creates an allocator holding a state written by pa_alloc_serialize (resume).  The bytes are checked
  * before use: format and version, every count against the buffer's length, every block id in the pool,
  * no block listed twice in the free list or the LRU, table lengths against request lengths, trie parents
- * present.  On any error nothing is created and *out is NULL.
+ * present; then the state's consistency: each block's refcount equals the number of request tables
+ * holding it, every unreferenced block is either free (unregistered) or parked in the LRU (registered),
+ * and each trie node's child count equals the nodes naming it as parent.  On any error nothing is created
+ * and *out is NULL.
  * Errors: INVALID_ARG, OOM. */
 pa_status pa_alloc_deserialize(const uint8_t* buf, size_t size, pa_alloc** out);
 

@@ -750,6 +750,29 @@ pa_status pa_alloc_deserialize(const uint8_t* buf, size_t size, pa_alloc** out) 
         a->in_lru[b] = 1;
     }
     if (!r.ok || r.n != size) return bad("length");
+    // Cross-checks, so that only a consistent state is accepted: a block's refcount is the number of
+    // request tables holding it; every unreferenced block is either free (unregistered) or parked
+    // (registered, in the LRU), and nothing else is; a node's child count is the number of nodes
+    // naming it as parent.
+    std::vector<int64_t> held(nb, 0);
+    for (const auto& kv : a->reqs)
+        for (int32_t b : kv.second.table) held[b] += 1;
+    int64_t unreferenced = 0;
+    for (int32_t b = 0; b < nb; ++b) {
+        if (held[b] != a->refcount[b]) return bad("refcount does not match the block tables");
+        unreferenced += a->refcount[b] == 0;
+    }
+    for (int32_t b : a->free_list)
+        if (a->refcount[b] != 0 || a->block_node[b] >= 0) return bad("free block in use or registered");
+    if (unreferenced != static_cast<int64_t>(a->free_list.size() + a->lru.size()))
+        return bad("unreferenced block neither free nor parked");
+    std::unordered_map<int64_t, int32_t> kids;
+    for (const auto& kv : a->node_key)
+        if (kv.second.parent != -1) kids[kv.second.parent] += 1;
+    for (const auto& kv : a->node_key) {
+        auto k = kids.find(kv.first);
+        if (a->children[kv.first] != (k == kids.end() ? 0 : k->second)) return bad("trie child count");
+    }
     *out = a;
     return PA_OK;
 }

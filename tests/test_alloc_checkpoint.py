@@ -112,3 +112,52 @@ def test_malformed_state_is_refused():
             pk.BlockAllocator.deserialize(bytes(bad)).close()
         except pk.PagedKVError:
             pass
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_every_reachable_state_is_accepted(seed):
+    """The consistency checks of the reader (refcounts against the tables, free and parked blocks,
+    child counts) hold in every state the operations reach: each one reads back to the same bytes."""
+    rng = np.random.default_rng(100 + seed)
+    bs = int(rng.choice([2, 4]))
+    a = pk.BlockAllocator(20, bs, free_order=rng.permutation(20))
+    for op in _run_ops(rng, 150, 20, bs):
+        _apply(a, op)
+        state = a.serialize()
+        b = pk.BlockAllocator.deserialize(state)
+        assert b.serialize() == state
+        b.close()
+
+
+# byte offset of the first free-list entry: magic, version, num_blocks, block_size (4 x 4 bytes), four i64
+# counters, the u64 free-list length; the refcounts follow the free list
+FREE_LIST_AT = 16 + 32 + 8
+
+
+def test_inconsistent_state_is_refused():
+    """Well-formed bytes that describe an impossible state are refused: a refcount that disagrees with
+    the block tables, and a block that is both free and held by a request."""
+    a = pk.BlockAllocator(12, 4)
+    assert a.allocate(1, 9) == pk.PA_OK                  # 3 blocks held
+    assert a.allocate(2, 4) == pk.PA_OK                  # 1 block held
+    good = a.serialize()
+    nf = len(a.free_list())
+    assert nf == 8
+    off = FREE_LIST_AT + 4 * nf                          # refcount[0]
+    st, table = a.get_block_table(1)
+    assert st == pk.PA_OK
+    held = int(table[0])
+    # one more reference than the tables hold
+    bad = bytearray(good)
+    rc = int.from_bytes(bad[off + 4 * held: off + 4 * held + 4], "little")
+    assert rc == 1
+    bad[off + 4 * held: off + 4 * held + 4] = (2).to_bytes(4, "little")
+    with pytest.raises(pk.PagedKVError):
+        pk.BlockAllocator.deserialize(bytes(bad))
+    # the top of the free stack replaced by a block that request 1 holds
+    bad = bytearray(good)
+    top = FREE_LIST_AT + 4 * (nf - 1)                    # the last free-list entry
+    bad[top: top + 4] = held.to_bytes(4, "little")
+    with pytest.raises(pk.PagedKVError):
+        pk.BlockAllocator.deserialize(bytes(bad))
+    pk.BlockAllocator.deserialize(good).close()           # the untouched bytes still read
