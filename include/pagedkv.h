@@ -19,6 +19,9 @@
  *   never synchronises.  Kernels are enqueued on `stream` (a cudaStream_t
  *   passed as void*; NULL = the legacy default stream) on the current device.
  *   Argument errors are detected on the host before anything is enqueued.
+ *   Pointers themselves are not inspected: one that is not memory of the
+ *   current device is the caller's error and faults the kernel that reads it
+ *   (the Python binding refuses host tensors and other devices' tensors).
  * - fp16 buffers (pa_half) hold IEEE-754 binary16 values.  Arithmetic inside
  *   the attention kernels is fp32; outputs are rounded to fp16 (nearest even).
  * - The KV cache is two separate tensors, K and V, each laid out

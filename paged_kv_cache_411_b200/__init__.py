@@ -346,6 +346,18 @@ def _need(cond, msg):
         raise PagedKVError(PA_ERR_INVALID_ARG, msg)
 
 
+def _on_device(*ts):
+    """The kernels dereference every pointer on the current device: refuse host tensors and tensors of
+    another GPU here, before the C call (the library itself does not inspect pointers)."""
+    import torch
+    ts = [t for t in ts if t is not None]
+    for t in ts:
+        _need(t.is_cuda, f"CUDA tensors expected; got one on {t.device}")
+    dev = torch.cuda.current_device()
+    for t in ts:
+        _need(t.device.index == dev, f"tensors must be on the current CUDA device (cuda:{dev}); got one on {t.device}")
+
+
 def reshape_and_cache(k_new, v_new, k_cache, v_cache, slot_mapping, err_flag=None, stream=None):
     """pa_reshape_and_cache on torch tensors: k_new/v_new [T,H,D] fp16, caches [NB,bs,H,D] fp16,
     slot_mapping [T] int64 (device)."""
@@ -353,6 +365,7 @@ def reshape_and_cache(k_new, v_new, k_cache, v_cache, slot_mapping, err_flag=Non
     _need(k_new.dtype == torch.float16 and k_cache.dtype == torch.float16, "fp16 tensors expected")
     _need(slot_mapping.dtype == torch.int64, "slot_mapping must be int64")
     _need(all(t.is_contiguous() for t in (k_new, v_new, k_cache, v_cache, slot_mapping)), "contiguous tensors expected")
+    _on_device(k_new, v_new, k_cache, v_cache, slot_mapping, err_flag)
     T, H, D = k_new.shape
     NB, bs = k_cache.shape[:2]
     check(lib().pa_reshape_and_cache(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping),
@@ -371,6 +384,7 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, sca
     _need(q.dtype == torch.float16 and out.dtype == torch.float16, "fp16 tensors expected")
     _need(block_tables.dtype == torch.int32 and seq_lens.dtype == torch.int32, "int32 tables expected")
     _need(all(t.is_contiguous() for t in (out, q, k_cache, v_cache, block_tables, seq_lens)), "contiguous tensors expected")
+    _on_device(out, q, k_cache, v_cache, block_tables, seq_lens, workspace, err_flag)
     S, H, D = q.shape
     NB, bs = k_cache.shape[:2]
     max_blocks = block_tables.shape[1] if block_tables.dim() == 2 else 0
@@ -388,6 +402,7 @@ def paged_attention_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_l
     _need(q.dtype == torch.float16 and out.dtype == torch.float16, "fp16 tensors expected")
     _need(block_tables.dtype == torch.int32 and seq_lens.dtype == torch.int32, "int32 tables expected")
     _need(all(t.is_contiguous() for t in (out, q, k_cache, v_cache, block_tables, seq_lens)), "contiguous tensors expected")
+    _on_device(out, q, k_cache, v_cache, block_tables, seq_lens, err_flag)
     S, H, D = q.shape
     NB, bs = k_cache.shape[:2]
     check(lib().pa_paged_attention_decode_noalloc(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
@@ -404,6 +419,7 @@ def paged_attention_prefill_chunk(out, q, k_cache, v_cache, block_tables, q_star
     _need(q.dtype == torch.float16 and out.dtype == torch.float16, "fp16 tensors expected")
     _need(all(t.is_contiguous() for t in (out, q, k_cache, v_cache, block_tables, q_start, ctx_before)),
           "contiguous tensors expected")
+    _on_device(out, q, k_cache, v_cache, block_tables, q_start, ctx_before, err_flag)
     T, H, D = q.shape
     NB, bs = k_cache.shape[:2]
     B = ctx_before.shape[0]

@@ -176,6 +176,26 @@ def test_cpp_allocator_matches_oracle_on_random_logs(N, bs, shuffled, log):
     _compare_state(ca, om, range(6))
 
 
+def test_binding_refuses_host_tensors():
+    """The kernel wrappers refuse tensors that are not on the GPU before any C call, since the kernels
+    would dereference them on the device."""
+    import torch
+    H, D, bs, nb = 4, 64, 16, 4
+    q = torch.zeros(1, H, D, dtype=torch.float16)
+    kc = torch.zeros(nb, bs, H, D, dtype=torch.float16)
+    tables = torch.zeros(1, 2, dtype=torch.int32)
+    lens = torch.ones(1, dtype=torch.int32)
+    with pytest.raises(pk.PagedKVError, match="CUDA tensors expected"):
+        pk.paged_attention_decode(q.clone(), q, kc, kc, tables, lens, 0.125, torch.zeros(1 << 12, dtype=torch.uint8))
+    with pytest.raises(pk.PagedKVError, match="CUDA tensors expected"):
+        pk.paged_attention_decode_noalloc(q.clone(), q, kc, kc, tables, lens, 0.125)
+    with pytest.raises(pk.PagedKVError, match="CUDA tensors expected"):
+        pk.paged_attention_prefill_chunk(q.clone(), q, kc, kc, tables, torch.tensor([0, 1], dtype=torch.int32),
+                                         torch.zeros(1, dtype=torch.int32), 0.125)
+    with pytest.raises(pk.PagedKVError, match="CUDA tensors expected"):
+        pk.reshape_and_cache(q, q, kc, kc, torch.zeros(1, dtype=torch.int64))
+
+
 def test_cpp_allocator_error_paths():
     with pytest.raises(pk.PagedKVError):
         pk.BlockAllocator(4, 16, [0, 1, 1, 2])
