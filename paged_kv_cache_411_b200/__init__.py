@@ -355,7 +355,7 @@ def _on_device(*ts):
         _need(t.is_cuda, f"CUDA tensors expected; got one on {t.device}")
     dev = torch.cuda.current_device()
     for t in ts:
-        _need(t.device.index == dev, f"tensors must be on the current CUDA device (cuda:{dev}); got one on {t.device}")
+        _need(t.get_device() == dev, f"tensors must be on the current CUDA device (cuda:{dev}); got one on {t.device}")
 
 
 def reshape_and_cache(k_new, v_new, k_cache, v_cache, slot_mapping, err_flag=None, stream=None):
