@@ -51,6 +51,22 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, FALLBACK_TFLOPS, "fallback"
 
 
+def packed_views(specs, make):
+    """One uint8 buffer holding a tensor per (name, shape, dtype) of ``specs``, each at a 256-byte aligned
+    offset, so that a step's inputs (or outputs) cross between host and device in ONE copy.  ``make(n)``
+    allocates the n-byte buffer; returns it and a typed, contiguous view per name."""
+    import torch
+    offs, n = {}, 0
+    for name, shape, dtype in specs:
+        nbytes = int(np.prod(shape, dtype=np.int64)) * torch.empty((), dtype=dtype).element_size()
+        offs[name] = (n, nbytes)
+        n = (n + nbytes + 255) // 256 * 256
+    buf = make(max(n, 256))
+    views = {name: buf[offs[name][0]:offs[name][0] + offs[name][1]].view(dtype).view(shape)
+             for name, shape, dtype in specs}
+    return buf, views
+
+
 def prefill_flops(w):
     """Algorithmic FLOPs of the causal chunk: 4 * H * D per visible (query, key) pair."""
     if w.prefill is None:
@@ -437,13 +453,22 @@ def run_ours(args):
     names = ("q", "k_step", "v_step", "slot_mapping", "block_tables", "seq_lens")
     if pout is not None:
         names += ("prefill_q", "prefill_table", "prefill_q_start", "prefill_ctx_before")
-    host = {k: getattr(ds, k).cpu().pin_memory() for k in names}
-    outs = [out] + ([pout] if pout is not None else [])
-    host_out = [[torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs] for _ in range(2)]
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = sum(t.numel() * t.element_size() for t in host_out[0])
-    dev_in = [{k: torch.empty_like(getattr(ds, k)) for k in names} for _ in range(2)]
-    dev_out = [[torch.empty_like(o) for o in outs] for _ in range(2)]
+    # every input of a step in one pinned buffer and every output in another (one copy each way per step,
+    # as the serving loop stages its tables, slots and lengths)
+    in_specs = [(k, tuple(getattr(ds, k).shape), getattr(ds, k).dtype) for k in names]
+    out_specs = [("out", tuple(out.shape), out.dtype)] + \
+        ([("pout", tuple(pout.shape), pout.dtype)] if pout is not None else [])
+    host_in, host_v = packed_views(in_specs, lambda n: torch.empty(n, dtype=torch.uint8).pin_memory())
+    for k in names:
+        host_v[k].copy_(getattr(ds, k).cpu())
+    host_out = [packed_views(out_specs, lambda n: torch.empty(n, dtype=torch.uint8).pin_memory())[0]
+                for _ in range(2)]
+    dev_sets = [packed_views(in_specs, lambda n: torch.empty(n, dtype=torch.uint8, device=device))
+                for _ in range(2)]
+    dev_outs = [packed_views(out_specs, lambda n: torch.empty(n, dtype=torch.uint8, device=device))
+                for _ in range(2)]
+    h2d = host_in.numel()
+    d2h = host_out[0].numel()
     copy_stream = torch.cuda.Stream(device)
     ready = [torch.cuda.Event() for _ in range(2)]      # inputs of the set are on the device
     done = [torch.cuda.Event() for _ in range(2)]       # the step that used the set has finished
@@ -452,26 +477,24 @@ def run_ours(args):
     def e2e_upload(b):
         with torch.cuda.stream(copy_stream):
             copy_stream.wait_event(done[b])              # the step before last has finished with set b
-            for k, t in host.items():
-                dev_in[b][k].copy_(t, non_blocking=True)
+            dev_sets[b][0].copy_(host_in, non_blocking=True)
             ready[b].record(copy_stream)
 
     def e2e_compute(b):
-        d = dev_in[b]
+        d, o = dev_sets[b][1], dev_outs[b][1]
         stream.wait_event(ready[b])
         pk.reshape_and_cache(d["k_step"], d["v_step"], ds.k_cache, ds.v_cache, d["slot_mapping"], stream=stream)
         if pout is not None:
-            pk.paged_attention_prefill_chunk(dev_out[b][1], d["prefill_q"], ds.k_cache, ds.v_cache,
+            pk.paged_attention_prefill_chunk(o["pout"], d["prefill_q"], ds.k_cache, ds.v_cache,
                                              d["prefill_table"], d["prefill_q_start"], d["prefill_ctx_before"],
                                              w.scale, stream=stream)
         if S > 0:
-            pk.paged_attention_decode(dev_out[b][0], d["q"], ds.k_cache, ds.v_cache, d["block_tables"],
+            pk.paged_attention_decode(o["out"], d["q"], ds.k_cache, ds.v_cache, d["block_tables"],
                                       d["seq_lens"], w.scale, ws, stream=stream)
         done[b].record(stream)
         with torch.cuda.stream(copy_stream):
             copy_stream.wait_event(done[b])
-            for h, dv in zip(host_out[b], dev_out[b]):
-                h.copy_(dv, non_blocking=True)
+            host_out[b].copy_(dev_outs[b][0], non_blocking=True)
             fetched[b].record(copy_stream)
 
     def e2e_run(n):

@@ -49,6 +49,36 @@ def test_prefill_8k_flops():
     assert bench.prefill_flops(w) == 4 * 32 * 128 * (8192 * 8193 // 2)
 
 
+def test_packed_views_stage_a_step_in_one_buffer():
+    """The end-to-end loop's staging: every tensor of a step in one buffer, 256-byte aligned, disjoint,
+    typed and contiguous, and a byte copy of the whole buffer carries every tensor."""
+    specs = [("q", (3, 4, 64), torch.float16), ("slots", (3,), torch.int64), ("tables", (3, 5), torch.int32),
+             ("empty", (0, 5), torch.int32), ("lens", (3,), torch.int32)]
+    buf, v = bench.packed_views(specs, lambda n: torch.zeros(n, dtype=torch.uint8))
+    base = buf.data_ptr()
+    spans = []
+    for name, shape, dtype in specs:
+        t = v[name]
+        assert tuple(t.shape) == shape and t.dtype == dtype and t.is_contiguous()
+        if t.numel() == 0:
+            continue                                   # an empty view may report a null pointer
+        assert (t.data_ptr() - base) % 256 == 0
+        spans.append((t.data_ptr() - base, t.numel() * t.element_size()))
+    spans.sort()
+    for (o0, n0), (o1, _) in zip(spans, spans[1:]):
+        assert o0 + n0 <= o1
+    assert spans[-1][0] + spans[-1][1] <= buf.numel()
+    g = torch.Generator().manual_seed(0)
+    v["q"].copy_(torch.randn(3, 4, 64, generator=g).half())
+    v["slots"].copy_(torch.tensor([7, -1, 2**40]))
+    v["tables"].copy_(torch.arange(15, dtype=torch.int32).view(3, 5))
+    v["lens"].copy_(torch.tensor([1, 2, 3], dtype=torch.int32))
+    buf2, v2 = bench.packed_views(specs, lambda n: torch.zeros(n, dtype=torch.uint8))
+    buf2.copy_(buf)
+    for name, _, _ in specs:
+        assert torch.equal(v2[name], v[name])
+
+
 def test_timing_distribution():
     d = bench.dist_ms([1.0, 2.0, 3.0, 4.0, 100.0])
     assert d["median"] == 3.0 and d["n"] == 5 and d["mean"] == 22.0
