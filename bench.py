@@ -393,23 +393,24 @@ def run_ours(args):
     dec_b, rs_b, pre_b = step_bytes(w, ds.seq_lens_host, ds.max_blocks, T)
     step_b = dec_b + rs_b + pre_b
 
-    def step(ev=None, pev=None):
-        pk.reshape_and_cache(ds.k_step, ds.v_step, ds.k_cache, ds.v_cache, ds.slot_mapping, stream=stream)
+    def step(ev=None, pev=None, st=None):
+        st = stream if st is None else st
+        pk.reshape_and_cache(ds.k_step, ds.v_step, ds.k_cache, ds.v_cache, ds.slot_mapping, stream=st)
         if pout is not None:
             if pev is not None:
-                pev[0].record(stream)
+                pev[0].record(st)
             pk.paged_attention_prefill_chunk(pout, ds.prefill_q, ds.k_cache, ds.v_cache, ds.prefill_table,
-                                             ds.prefill_q_start, ds.prefill_ctx_before, w.scale, stream=stream)
+                                             ds.prefill_q_start, ds.prefill_ctx_before, w.scale, stream=st)
             if pev is not None:
-                pev[1].record(stream)
+                pev[1].record(st)
         if S == 0:
             return
         if ev is not None:
-            ev[0].record(stream)
+            ev[0].record(st)
         pk.paged_attention_decode(out, ds.q, ds.k_cache, ds.v_cache, ds.block_tables, ds.seq_lens, w.scale, ws,
-                                  stream=stream)
+                                  stream=st)
         if ev is not None:
-            ev[1].record(stream)
+            ev[1].record(st)
 
     for _ in range(args.warmup):
         step()
@@ -520,6 +521,34 @@ def run_ours(args):
     e2e_max, e2e_bytes = reduce_max_sum(e2e_s, step_b * args.steps, device)
     e2e_value = e2e_bytes / e2e_max / 1e9
 
+    # the same step captured once in a CUDA graph and replayed: the kernels and their programmatic-launch
+    # edges as above, without the host's per-launch cost (1 GPU; reported beside the stream-launched step)
+    graph = None
+    if world == 1 and not args.no_graph:
+        try:
+            g = torch.cuda.CUDAGraph()
+            cap = torch.cuda.Stream(device)               # capture needs a stream other than the default one
+            torch.cuda.synchronize(device)
+            with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
+                step(st=cap)
+            with torch.cuda.stream(stream):
+                for _ in range(args.warmup):
+                    g.replay()
+                g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                torch.cuda.synchronize(device)
+                g0.record(stream)
+                for _ in range(args.steps):
+                    g.replay()
+                g1.record(stream)
+            torch.cuda.synchronize(device)
+            g_ms = g0.elapsed_time(g1) / args.steps
+            graph = {"value": round(step_b / (g_ms / 1e3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(g_ms, 5),
+                     "steps": args.steps}
+            del g
+        except Exception as exc:                     # reported, not fatal: the stream-launched figures stand
+            torch.cuda.synchronize(device)
+            graph = {"error": f"{type(exc).__name__}: {exc}"[:200]}
+
     if rank == 0:
         has_decode = S > 0
         dec_avg_ms = float(np.mean(dec_ms)) if has_decode else 0.0
@@ -548,6 +577,7 @@ def run_ours(args):
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": round(1e3 * e2e_max / args.steps, 4)},
             "gpu_launches": args.steps * (1 + (3 if S > 0 else 0) + (1 if pout is not None else 0)),
+            "graph": graph,
             "kv_pool": pool_stats(ds),
             "clocks": clk.summary(),
         }
@@ -762,6 +792,7 @@ def main(argv=None):
     ap.add_argument("--oracle-tokens", type=int, default=40000,
                     help="cached tokens in the cpu_baseline leg's bounded sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay of the step")
     ap.add_argument("--serve", action="store_true",
                     help="continuous-batching run over a seeded trace instead of the single-step benchmark")
     ap.add_argument("--serve-requests", type=int, default=1000)
