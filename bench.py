@@ -11,6 +11,10 @@ over ranks.  With N > 1 (torchrun) every rank runs its own replica of the
 workload on its own GPU (weak scaling, no collective on the data path); the
 time is the max over ranks.
 
+At N = 1 the line also carries ``graph``: the same step captured once in a
+CUDA graph and replayed (and the decode call alone), which takes the host's
+per-call launch path out of the timing; ``--no-graph`` skips it.
+
 ``--impl reference`` times the float64 CPU oracle on the host cores instead
 (a bounded sample of the same workload per step); under torchrun only rank 0
 runs it.
