@@ -5,7 +5,6 @@ import io
 import json
 import os
 import socket
-import sys
 from contextlib import redirect_stdout
 
 import numpy as np

@@ -2,7 +2,6 @@
 shared system-prompt example, then the C++ allocator against the oracle, bit for bit, on
 random logs of prefix-sharing requests (no GPU)."""
 import numpy as np
-import pytest
 from hypothesis import given, settings
 from hypothesis import strategies as st
 
