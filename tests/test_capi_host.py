@@ -36,6 +36,25 @@ def test_library_exports_every_declared_symbol():
     assert lib.pa_abi_version() == 2
 
 
+def test_header_serves_a_plain_c_program(tmp_path):
+    """include/pagedkv.h compiles as strict C11 and a C program linked against libpagedkv.so follows a
+    hand-traced allocator sequence (tests/c_consumer/alloc_from_c.c) with no Python in between."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = os.path.join(ROOT, "tests", "c_consumer", "alloc_from_c.c")
+    exe = str(tmp_path / "alloc_from_c")
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    r = subprocess.run([cc, "-std=c11", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        src, "-o", exe, "-L", libdir, "-lpagedkv", f"-Wl,-rpath,{libdir}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout + r.stderr
+
+
 def test_status_strings_and_device_flag():
     lib = pk.lib()
     assert lib.pa_status_string(pk.PA_ERR_OOM) == b"PA_ERR_OOM"
